@@ -1,0 +1,79 @@
+/*
+ * Oracle for exact scaled dot-product attention: TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, obviously correct CPU code in double precision.  Only the test
+ * suite, the smoke check and the benchmark's CPU-baseline leg may load it; the
+ * product library never does, and the two share no code.
+ *
+ * What it computes (the definition the attention pages derive from):
+ *   Attention(Q, K, V) = softmax(Q K^T * scale) V, softmax taken row by row
+ *   in its numerically stable, max-subtracted form
+ *   ("Attention at the Theoretical Minimum: A Mathematics of Arrays Framework
+ *   for Memory-Optimal Transformer Kernels", abstract; the agents-report.net
+ *   MoA article, section "DNF derivation", where scale = 1/sqrt(d_k)).
+ *
+ * For one query row i of one (batch, head) slice:
+ *   allowed(i, j) = true                          non-causal
+ *                 = j <= i + (n_kv - n_q)         causal (bottom-right aligned)
+ *   s_ij  = scale * sum_k Q[i,k] K[j,k]           (allowed j only)
+ *   m_i   = max_j s_ij
+ *   e_ij  = exp(s_ij - m_i),  l_i = sum_j e_ij
+ *   O[i,:] = (sum_j e_ij V[j,:]) / l_i
+ *   LSE_i = m_i + ln l_i                          (natural log of the scaled logits)
+ * A row with no allowed key gives O = 0 and LSE = -inf.
+ *
+ * Layout: row-major.  Q [n_q, d_k], K [n_kv, d_k], V [n_kv, d_v] per slice,
+ * slices back to back ([bh, n, d]).  Inputs are float32: every bf16 and fp32
+ * input value is exact in float32 and is widened exactly to double here.
+ *
+ * Parity pins: see tests/test_oracle_pins.py (closed forms, invariants, brute
+ * force, a hand-worked example and a library special case).
+ */
+#ifndef SDPA_ORACLE_H
+#define SDPA_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Full score matrix of one slice: S[i, j] = scale * q_i . k_j for allowed (i, j), -inf otherwise.
+   S is [n_q, n_kv].  Returns 0 or -1 on a bad argument. */
+int oracle_scores(const float* Q, const float* K, int64_t n_q, int64_t n_kv, int d_k, double scale,
+                  int causal, double* S);
+
+/* Row-wise softmax of an explicit matrix with the row maximum subtracted first.
+   Entries equal to -inf get probability 0; a row that is all -inf becomes all zeros. */
+int oracle_softmax_rows(const double* S, int64_t rows, int64_t cols, double* P);
+
+/* The naive, unstable softmax exp(s) / sum exp(s) with NO max subtraction.
+   Brute-force cross-check for small, well-scaled inputs only: it overflows for large logits. */
+int oracle_softmax_naive(const double* S, int64_t rows, int64_t cols, double* P);
+
+/* Full-matrix form for tiny problems: S (full), P = softmax_rows(S), O = P V, LSE.
+   S_out and P_out may be NULL.  O is [n_q, d_v], LSE is [n_q]. */
+int oracle_sdpa_full(const float* Q, const float* K, const float* V, int64_t n_q, int64_t n_kv, int d_k,
+                     int d_v, double scale, int causal, double* S_out, double* P_out, double* O,
+                     double* LSE);
+
+/* Row-at-a-time form over bh independent slices, for the listed query rows of every slice.
+   rows: n_rows indices in [0, n_q); NULL means all rows (n_rows must then equal n_q).
+   O is [bh, n_rows, d_v], LSE is [bh, n_rows].  threads <= 0 means 1. */
+int oracle_sdpa_rows(const float* Q, const float* K, const float* V, int64_t bh, int64_t n_q,
+                     int64_t n_kv, int d_k, int d_v, double scale, int causal, const int64_t* rows,
+                     int64_t n_rows, double* O, double* LSE, int threads);
+
+/* Decode: one query row per (b, h) against the first lens[b] keys of a cache.
+   Q [B, H, d_k]; K [B, H, n_cap, d_k]; V [B, H, n_cap, d_v]; O [B, H, d_v]; LSE [B, H].
+   Only the (b, h) pairs listed in `pairs` (flat b*H + h, n_pairs of them) are computed, into
+   O[p], LSE[p] in list order; pairs == NULL means all B*H pairs in order. */
+int oracle_decode(const float* Q, const float* K, const float* V, const int32_t* lens, int64_t B,
+                  int64_t H, int64_t n_cap, int d_k, int d_v, double scale, const int64_t* pairs,
+                  int64_t n_pairs, double* O, double* LSE, int threads);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif

@@ -1,0 +1,267 @@
+"""Pins for the CPU oracle: checks against facts fixed by the definition, not by the oracle itself.
+
+The method is exact attention, Attention(Q,K,V) = softmax(Q K^T * scale) V with
+a numerically stable (max-subtracted) softmax, derived with no intermediate
+arrays ("Attention at the Theoretical Minimum: A Mathematics of Arrays
+Framework for Memory-Optimal Transformer Kernels", abstract; agents-report.net
+MoA article, sections "DNF derivation" and "numerical verification").  The
+pages print no worked numbers, so the pins are closed forms, invariants,
+special cases that reduce to a library routine, and brute force.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(12345)
+
+
+def _frac(s):
+    return float(Fraction(s))
+
+
+def _ln(s):
+    assert s.startswith("ln ")
+    return math.log(float(s[3:]))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_worked_example_closed_form(causal):
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    q = np.array(g["Q"], np.float32)
+    k = np.array(g["K"], np.float32)
+    v = np.array(g["V"], np.float32)
+    exp = g["causal" if causal else "noncausal"]
+    O_exp = np.array([[_frac(x) for x in row] for row in exp["O"]])
+    L_exp = np.array([_ln(x) for x in exp["LSE"]])
+    for O, L in (oracle.sdpa_rows(q, k, v, math.log(2.0), causal), oracle.sdpa_full(q, k, v, math.log(2.0), causal)[:2]):
+        np.testing.assert_allclose(O, O_exp, rtol=0, atol=1e-15)
+        np.testing.assert_allclose(L, L_exp, rtol=0, atol=1e-15)
+    # the score matrix itself: scale * Q K^T, not K Q^T
+    S = oracle.scores(q, k, math.log(2.0), causal)
+    dots = np.array(g["dots"], np.float64) * math.log(2.0)
+    if causal:
+        dots[0, 2] = -np.inf
+    np.testing.assert_array_equal(S, dots)
+
+
+def test_single_key_returns_v_exactly():
+    # n_kv = 1: the only weight is exp(0)/exp(0) = 1, so O = V[0] bit for bit and LSE = s_00.
+    q = RNG.integers(-4, 5, size=(6, 16)).astype(np.float32)
+    k = RNG.integers(-4, 5, size=(1, 16)).astype(np.float32)
+    v = RNG.standard_normal((1, 8)).astype(np.float32)
+    O, L = oracle.sdpa_rows(q, k, v, 0.25)
+    np.testing.assert_array_equal(O, np.broadcast_to(v.astype(np.float64), O.shape))
+    dots = (q.astype(np.int64) @ k.astype(np.int64).T)[:, 0]  # exact integer dot products
+    np.testing.assert_array_equal(L, 0.25 * dots.astype(np.float64))
+
+
+def test_causal_first_row_is_v0():
+    n, d = 9, 8
+    q, k, v = (RNG.standard_normal((n, d)).astype(np.float32) for _ in range(3))
+    O, L = oracle.sdpa_rows(q, k, v, 0.3, causal=True)
+    np.testing.assert_array_equal(O[0], v[0].astype(np.float64))
+    S = oracle.scores(q[:1], k[:1], 0.3)
+    assert L[0] == S[0, 0]
+
+
+def test_constant_v_gives_constant_output():
+    n_q, n_kv, d = 7, 11, 5
+    q, k = RNG.standard_normal((n_q, d)).astype(np.float32), RNG.standard_normal((n_kv, d)).astype(np.float32)
+    row = RNG.standard_normal(6).astype(np.float32)
+    v = np.tile(row, (n_kv, 1))
+    for causal in (False, True):
+        O, _ = oracle.sdpa_rows(q, k, v, 0.7, causal)
+        np.testing.assert_allclose(O, np.broadcast_to(row.astype(np.float64), O.shape), rtol=4e-16, atol=0)
+
+
+def test_softmax_rows_sum_to_one_and_identity_v():
+    n, d = 12, 12
+    q, k = RNG.standard_normal((n, 8)).astype(np.float32), RNG.standard_normal((n, 8)).astype(np.float32)
+    for causal in (False, True):
+        S = oracle.scores(q, k, 0.9, causal)
+        P = oracle.softmax_rows(S)
+        np.testing.assert_allclose(P.sum(1), 1.0, rtol=0, atol=1e-15)
+        assert (P >= 0).all()
+        # V = I (n_kv = d_v) turns the output into the probability matrix itself
+        O, _ = oracle.sdpa_rows(q, k, np.eye(n, d, dtype=np.float32), 0.9, causal)
+        np.testing.assert_allclose(O, P, rtol=0, atol=1e-15)
+        np.testing.assert_allclose(O.sum(1), 1.0, rtol=0, atol=1e-15)
+        if causal:
+            assert (O[np.triu_indices(n, 1)] == 0).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_logits_give_mean_of_allowed_rows(causal):
+    n_q, n_kv, d = 6, 9, 4
+    q = RNG.standard_normal((n_q, d)).astype(np.float32)
+    k = RNG.standard_normal((n_kv, d)).astype(np.float32)
+    v = RNG.standard_normal((n_kv, 5)).astype(np.float32)
+    for qq, scale in ((np.zeros_like(q), 0.5), (q, 0.0)):
+        O, L = oracle.sdpa_rows(qq, k, v, scale, causal)
+        for i in range(n_q):
+            cnt = (i + n_kv - n_q + 1) if causal else n_kv
+            np.testing.assert_allclose(O[i], v[:cnt].astype(np.float64).mean(0), rtol=1e-14, atol=1e-15)
+            assert abs(L[i] - math.log(cnt)) < 1e-15
+
+
+def test_permutation_equivariance():
+    n_q, n_kv, d = 5, 13, 8
+    q = RNG.standard_normal((n_q, d)).astype(np.float32)
+    k = RNG.standard_normal((n_kv, d)).astype(np.float32)
+    v = RNG.standard_normal((n_kv, 6)).astype(np.float32)
+    O, L = oracle.sdpa_rows(q, k, v, 0.4)
+    perm = RNG.permutation(n_kv)
+    O2, L2 = oracle.sdpa_rows(q, k[perm], v[perm], 0.4)
+    np.testing.assert_allclose(O2, O, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(L2, L, rtol=0, atol=1e-14)
+    # permuting V alone must change the answer (the pairing of k_j with v_j matters)
+    O3, _ = oracle.sdpa_rows(q, k, v[perm], 0.4)
+    assert np.abs(O3 - O).max() > 1e-3
+
+
+def test_shift_invariance():
+    # K' = K + 1 u^T adds scale*(q_i . u) to every logit of row i: O unchanged, LSE shifted.
+    n_q, n_kv, d = 4, 10, 8
+    q = RNG.integers(-3, 4, size=(n_q, d)).astype(np.float32)
+    k = RNG.integers(-3, 4, size=(n_kv, d)).astype(np.float32)
+    u = RNG.integers(-5, 6, size=(d,)).astype(np.float32)
+    v = RNG.standard_normal((n_kv, 7)).astype(np.float32)
+    scale = 0.125
+    for causal in (False, True):
+        O, L = oracle.sdpa_rows(q, k, v, scale, causal)
+        O2, L2 = oracle.sdpa_rows(q, k + u, v, scale, causal)
+        shift = scale * (q.astype(np.int64) @ u.astype(np.int64)).astype(np.float64)
+        np.testing.assert_allclose(O2, O, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(L2, L + shift, rtol=0, atol=1e-12)
+
+
+def _brute_force(q, k, v, scale, causal):
+    """Independent pure-Python evaluation of the naive formula exp(s)/sum exp(s) (no max subtraction)."""
+    n_q, n_kv = len(q), len(k)
+    O, L = [], []
+    for i in range(n_q):
+        ws = []
+        for j in range(n_kv):
+            if causal and j > i + (n_kv - n_q):
+                ws.append(0.0)
+                continue
+            s = scale * math.fsum(float(a) * float(b) for a, b in zip(q[i], k[j]))
+            ws.append(math.exp(s))
+        z = math.fsum(ws)
+        O.append([math.fsum(w * float(v[j][c]) for j, w in enumerate(ws)) / z for c in range(len(v[0]))])
+        L.append(math.log(z))
+    return np.array(O), np.array(L)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n_q,n_kv,d_k,d_v", [(1, 1, 1, 1), (3, 5, 4, 2), (8, 8, 6, 3), (5, 8, 2, 7)])
+def test_brute_force_tiny(n_q, n_kv, d_k, d_v, causal):
+    q = RNG.uniform(-1, 1, (n_q, d_k)).astype(np.float32)
+    k = RNG.uniform(-1, 1, (n_kv, d_k)).astype(np.float32)
+    v = RNG.standard_normal((n_kv, d_v)).astype(np.float32)
+    scale = 1.3  # |s| < 5
+    O, L = oracle.sdpa_rows(q, k, v, scale, causal)
+    Ob, Lb = _brute_force(q, k, v, scale, causal)
+    np.testing.assert_allclose(O, Ob, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(L, Lb, rtol=0, atol=1e-13)
+    S = oracle.scores(q, k, scale, causal)
+    np.testing.assert_allclose(oracle.softmax_rows(S), oracle.softmax_naive(S), rtol=1e-13, atol=1e-15)
+
+
+def test_stability_large_logits():
+    # s = [800, 799, 798]: exp(800) overflows, the max-subtracted form gives weights 1 : e^-1 : e^-2.
+    q = np.array([[1.0]], np.float32)
+    k = np.array([[800.0], [799.0], [798.0]], np.float32)
+    v = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]], np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        naive = oracle.softmax_naive(oracle.scores(q, k, 1.0))
+    assert not np.isfinite(naive).all()
+    O, L = oracle.sdpa_rows(q, k, v, 1.0)
+    z = 1 + math.exp(-1) + math.exp(-2)
+    np.testing.assert_allclose(O[0], [(1 + math.exp(-2)) / z, (math.exp(-1) + math.exp(-2)) / z], rtol=1e-15)
+    assert abs(L[0] - (800 + math.log(z))) < 1e-12
+
+
+def test_causal_alignment_rectangular():
+    # bottom-right alignment: row i sees keys j <= i + (n_kv - n_q)
+    d = 4
+    q = RNG.standard_normal((3, d)).astype(np.float32)
+    k = RNG.standard_normal((2, d)).astype(np.float32)
+    v = RNG.standard_normal((2, 3)).astype(np.float32)
+    O, L = oracle.sdpa_rows(q, k, v, 0.5, causal=True)
+    assert (O[0] == 0).all() and L[0] == -np.inf          # no allowed key
+    np.testing.assert_array_equal(O[1], v[0].astype(np.float64))  # only key 0
+    Of, Lf = oracle.sdpa_rows(q, k, v, 0.5, causal=False)
+    np.testing.assert_allclose(O[2], Of[2], rtol=0, atol=1e-15)   # last row sees everything
+    # a single query row (decode) is unaffected by the causal flag
+    k5 = RNG.standard_normal((5, d)).astype(np.float32)
+    v5 = RNG.standard_normal((5, 3)).astype(np.float32)
+    a = oracle.sdpa_rows(q[:1], k5, v5, 0.5, causal=True)
+    b = oracle.sdpa_rows(q[:1], k5, v5, 0.5, causal=False)
+    np.testing.assert_array_equal(a[0], b[0])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_library_special_case_torch_float64(causal):
+    # Mirrors the pages' check of the DNF against PyTorch in double precision.
+    import torch
+    import seeded_inputs as si
+    n, d = 128, 64
+    q, k, v = (si.fill_host((1, 1, n, d), 0, s, bf16=False) for s in (0, 1, 2))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(x).double() for x in (q, k, v)), is_causal=causal, scale=1 / 8).numpy()
+    O, _ = oracle.sdpa_rows(q, k, v, 1 / 8, causal)
+    np.testing.assert_allclose(O, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_rows_subset_and_slices_match_full():
+    bh, n_q, n_kv, d = 3, 20, 17, 8
+    q = RNG.standard_normal((bh, n_q, d)).astype(np.float32)
+    k = RNG.standard_normal((bh, n_kv, d)).astype(np.float32)
+    v = RNG.standard_normal((bh, n_kv, 5)).astype(np.float32)
+    rows = np.array([0, 3, 19, 7])
+    for causal in (False, True):
+        O, L = oracle.sdpa_rows(q, k, v, 0.3, causal, rows=rows, threads=3)
+        for b in range(bh):
+            Of, Lf, _, _ = oracle.sdpa_full(q[b], k[b], v[b], 0.3, causal)
+            np.testing.assert_allclose(O[b], Of[rows], rtol=1e-14, atol=1e-15)
+            np.testing.assert_allclose(L[b], Lf[rows], rtol=1e-14, atol=1e-15)
+
+
+def test_decode_uses_only_first_len_keys():
+    B, H, n_cap, d = 3, 2, 16, 8
+    q = RNG.standard_normal((B, H, d)).astype(np.float32)
+    k = RNG.standard_normal((B, H, n_cap, d)).astype(np.float32)
+    v = RNG.standard_normal((B, H, n_cap, d)).astype(np.float32)
+    lens = np.array([1, 16, 7], np.int32)
+    for b in range(B):
+        k[b, :, lens[b]:] = np.nan
+        v[b, :, lens[b]:] = np.nan
+    O, L = oracle.decode(q, k, v, lens, 0.35)
+    assert np.isfinite(O).all() and np.isfinite(L).all()
+    for b in range(B):
+        for h in range(H):
+            n = lens[b]
+            Or, Lr = oracle.sdpa_rows(q[b, h][None], k[b, h, :n], v[b, h, :n], 0.35)
+            np.testing.assert_array_equal(O[b * H + h], Or[0])
+            assert L[b * H + h] == Lr[0]
+    np.testing.assert_array_equal(O[0], v[0, 0, 0].astype(np.float64))  # len 1 -> V[0]
+    pairs = np.array([5, 0])
+    Op, Lp = oracle.decode(q, k, v, lens, 0.35, pairs=pairs)
+    np.testing.assert_array_equal(Op, O[pairs])
+
+
+def test_rejects_bad_arguments():
+    q = np.zeros((2, 4), np.float32)
+    with pytest.raises(ValueError):
+        oracle.sdpa_rows(q, q, q, 1.0, rows=np.array([2]))
+    with pytest.raises(ValueError):
+        oracle.decode(np.zeros((1, 1, 4), np.float32), np.zeros((1, 1, 4, 4), np.float32),
+                      np.zeros((1, 1, 4, 4), np.float32), np.array([5], np.int32), 1.0)
