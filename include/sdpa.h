@@ -1,0 +1,131 @@
+/*
+ * sdpa.h -- C ABI of the B200 (sm_100a) exact scaled dot-product attention library.
+ *
+ * What every entry point computes, for each (batch b, head h) slice:
+ *
+ *     O = softmax(Q K^T * scale) V          (row-wise, numerically stable softmax)
+ *     LSE_i = ln sum_j exp(scale * q_i . k_j)   over the keys row i may see
+ *
+ * This is the attention definition of the Mathematics-of-Arrays article
+ * (agents-report.net, "DNF derivation": Attention(Q,K,V) = softmax(QK^T/sqrt(d_k))V,
+ * here with the scale passed in) and of the MoA paper's abstract ("Attention at
+ * the Theoretical Minimum", paperdance.org): no intermediate array -- no n x n
+ * score or probability buffer and no transposed-key copy -- is ever written to
+ * memory, so global-memory traffic is O(n*d_k + n*d_v): Q, K and V are read and
+ * O (and LSE) written, once.
+ *
+ * Conventions shared by all entry points
+ *  - Layout: row-major and contiguous.  Q [batch, heads, n_q, d_k],
+ *    K [batch, heads, n_kv, d_k], V [batch, heads, n_kv, d_v],
+ *    O [batch, heads, n_q, d_v], LSE [batch, heads, n_q] (float).
+ *  - Ownership: every pointer is caller-owned DEVICE memory, valid until the work
+ *    queued on `stream` has finished.  The library allocates no memory.
+ *  - Execution: asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) on the current device.  No call synchronises except
+ *    sdpa_get_last_device_error.
+ *  - Causal masking is bottom-right aligned: query row i sees key j iff
+ *    j <= i + (n_kv - n_q).  A row that sees no key (only when n_q > n_kv) gets
+ *    O = 0 and LSE = -inf.
+ *  - LSE may be NULL (not written).  It is the natural log of the SCALED logits.
+ *  - Errors: argument checks run on the host before any launch and return a
+ *    status without touching memory.  A failed launch returns SDPA_ERR_CUDA.
+ *    Problems found on the device (a pipeline wait that ran out of time, a decode
+ *    length outside [1, n_kv_cap]) set a device error word that
+ *    sdpa_get_last_device_error reads; kernels never trap.
+ *  - Degenerate shapes: batch == 0, heads == 0 or n_q == 0 -> SDPA_OK, nothing written.
+ */
+#ifndef SDPA_B200_H
+#define SDPA_B200_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define SDPA_API __attribute__((visibility("default")))
+#else
+#define SDPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SDPA_OK = 0,
+  SDPA_ERR_INVALID_ARG = 1,     /* null pointer, negative size, n_kv == 0, bad flag */
+  SDPA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. head dim) */
+  SDPA_ERR_MISALIGNED = 3,      /* a pointer is not 16-byte aligned */
+  SDPA_ERR_WORKSPACE = 4,       /* workspace missing or too small */
+  SDPA_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed */
+  SDPA_ERR_DEVICE_TIMEOUT = 6,  /* a kernel pipeline wait gave up (device error word) */
+  SDPA_ERR_DEVICE_BAD_LENGTH = 7 /* a decode length was outside [1, n_kv_cap] (device error word) */
+} sdpa_status;
+
+/*
+ * sdpa_fwd -- bf16 prefill on the 5th-generation tensor cores (tcgen05/TMEM, TMA).
+ *
+ * Q, K, V, O: __nv_bfloat16, layout above.  LSE: float or NULL.
+ * d_k == d_v, and both in {64, 128} (else SDPA_ERR_UNSUPPORTED).
+ * n_q >= 0, n_kv >= 1.  batch*heads*max(n_q, n_kv) < 2^31.
+ * causal: 0 or 1.  scale: finite (else SDPA_ERR_INVALID_ARG) and > 0 (else
+ * SDPA_ERR_UNSUPPORTED; the online softmax tracks the row maximum of the raw
+ * scores, which is the maximum of the scaled ones only for a positive scale).
+ * Every pointer 16-byte aligned (TMA), else SDPA_ERR_MISALIGNED.
+ * Arithmetic: S = Q K^T and O += P V on the tensor cores with fp32
+ * accumulation; softmax in fp32 with P rounded to bf16; O rounded to bf16
+ * (round to nearest even); LSE in fp32.
+ */
+SDPA_API int sdpa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int batch, int heads,
+             int n_q, int n_kv, int d_k, int d_v, float scale, int causal, void* stream);
+
+/*
+ * sdpa_fwd_f32 -- fp32 prefill on the CUDA cores (FMA pipes); same semantics as
+ * sdpa_fwd with float tensors.  1 <= d_k, d_v <= 128.  Scores, softmax
+ * weights and the output sum are all fp32 (no tensor cores: TF32 would lose
+ * about three decimal digits).  Pointers must be 4-byte aligned.
+ */
+SDPA_API int sdpa_fwd_f32(const float* Q, const float* K, const float* V, float* O, float* LSE, int batch,
+                 int heads, int n_q, int n_kv, int d_k, int d_v, float scale, int causal, void* stream);
+
+/*
+ * sdpa_decode_workspace_size -- bytes of device workspace sdpa_decode needs
+ * for this shape (partial outputs and log-sum-exps of the KV splits).
+ * Returns 0 for a degenerate or invalid shape.
+ */
+SDPA_API size_t sdpa_decode_workspace_size(int batch, int heads, int n_kv_cap, int d_v);
+
+/*
+ * sdpa_decode -- one query row per (batch, head) against a KV cache (split-KV).
+ *
+ * Q [batch, heads, d_k]; K [batch, heads, n_kv_cap, d_k]; V [batch, heads, n_kv_cap, d_v],
+ * all __nv_bfloat16.  kv_lens: int32 [batch] in DEVICE memory, each in
+ * [1, n_kv_cap]: sequence b attends to cache rows 0 .. kv_lens[b]-1, and rows
+ * at or past kv_lens[b] are never read (they may hold anything, NaN included).
+ * O [batch, heads, d_v] bf16; LSE [batch, heads] float or NULL.
+ * d_k == d_v in {64, 128}.  All pointers 16-byte aligned.
+ * workspace: caller-owned device memory of at least
+ * sdpa_decode_workspace_size(batch, heads, n_kv_cap, d_v) bytes, else
+ * SDPA_ERR_WORKSPACE; its contents need no initialisation and are scratch
+ * afterwards.  A length outside [1, n_kv_cap] is clamped on the device and
+ * reported as SDPA_ERR_DEVICE_BAD_LENGTH by sdpa_get_last_device_error.
+ * (A single query row sees every cached key, so causal masking does not apply.)
+ */
+SDPA_API int sdpa_decode(const void* Q, const void* K, const void* V, const int* kv_lens, void* O, float* LSE,
+                int batch, int heads, int n_kv_cap, int d_k, int d_v, float scale, void* workspace,
+                size_t workspace_bytes, void* stream);
+
+/*
+ * sdpa_get_last_device_error -- synchronise `stream`, then read and clear the
+ * device error word of the current device.  Returns SDPA_OK, the first device
+ * error recorded since the last call, or SDPA_ERR_CUDA if the synchronisation
+ * itself failed.
+ */
+SDPA_API int sdpa_get_last_device_error(void* stream);
+
+/* sdpa_status_string -- a static, human-readable name for a status code. */
+SDPA_API const char* sdpa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDPA_B200_H */

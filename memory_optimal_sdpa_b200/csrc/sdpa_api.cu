@@ -1,0 +1,208 @@
+// sdpa_api.cu -- the C ABI (include/sdpa.h): argument checks, TMA tensor-map
+// encoding and kernel launches.  One translation unit holds every kernel so the
+// device error word is a single symbol without relocatable device code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "sdpa.h"
+#include "prefill_bf16.cuh"
+#include "prefill_f32.cuh"
+#include "decode.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [bh][n][d] bf16 tensor, 64-column x 128-row boxes, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* ptr, int d, int n, int bh) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)bh};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+bool aligned4(const void* p) { return ((uintptr_t)p & 3u) == 0; }
+
+// The current device must be an sm_100 part (B200 class).
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SDPA_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return SDPA_ERR_CUDA;
+  if (major != 10 || minor != 0) return SDPA_ERR_UNSUPPORTED;
+  return SDPA_OK;
+}
+
+template <int D, bool CAUSAL>
+int launch_prefill(const void* Q, const void* K, const void* V, void* O, float* LSE, int bh, int n_q,
+                   int n_kv, float scale, cudaStream_t stream) {
+  using Cfg = sdpa::PrefillCfg<D>;
+  auto kern = sdpa::sdpa_fwd_bf16_kernel<D, CAUSAL>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return SDPA_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, D, n_q, bh) || !make_map(&mk, K, D, n_kv, bh) || !make_map(&mv, V, D, n_kv, bh))
+    return SDPA_ERR_CUDA;
+  sdpa::PrefillParams p;
+  p.O = (__nv_bfloat16*)O;
+  p.LSE = LSE;
+  p.n_q = n_q;
+  p.n_kv = n_kv;
+  p.bh_count = bh;
+  p.n_pairs = (n_q + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long grid = (long long)bh * p.n_pairs;
+  kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+size_t decode_ws_bytes(long long batch, long long heads, long long n_cap, long long d_v) {
+  const long long chunk = sdpa::decode_chunk(batch, heads, n_cap);
+  const long long ns = (n_cap + chunk - 1) / chunk;
+  return (size_t)(batch * heads * ns) * (size_t)(d_v + 1) * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" int sdpa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int batch,
+                        int heads, int n_q, int n_kv, int d_k, int d_v, float scale, int causal,
+                        void* stream) {
+  if (batch < 0 || heads < 0 || n_q < 0 || n_kv < 1 || (causal != 0 && causal != 1) || !std::isfinite(scale))
+    return SDPA_ERR_INVALID_ARG;
+  if (d_k != d_v || (d_k != 64 && d_k != 128) || !(scale > 0.f)) return SDPA_ERR_UNSUPPORTED;
+  if (batch == 0 || heads == 0 || n_q == 0) return SDPA_OK;
+  if (!Q || !K || !V || !O) return SDPA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (LSE && !aligned4(LSE)))
+    return SDPA_ERR_MISALIGNED;
+  const long long bh = (long long)batch * heads;
+  if (bh * (long long)(n_q > n_kv ? n_q : n_kv) >= (1LL << 31) || bh * ((n_q + 255) / 256) >= (1LL << 31))
+    return SDPA_ERR_UNSUPPORTED;
+  if (int e = check_device()) return e;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (d_k == 64)
+    return causal ? launch_prefill<64, true>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, s)
+                  : launch_prefill<64, false>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, s);
+  return causal ? launch_prefill<128, true>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, s)
+                : launch_prefill<128, false>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, s);
+}
+
+extern "C" int sdpa_fwd_f32(const float* Q, const float* K, const float* V, float* O, float* LSE, int batch,
+                            int heads, int n_q, int n_kv, int d_k, int d_v, float scale, int causal,
+                            void* stream) {
+  if (batch < 0 || heads < 0 || n_q < 0 || n_kv < 1 || d_k < 1 || d_v < 1 || (causal != 0 && causal != 1) ||
+      !std::isfinite(scale))
+    return SDPA_ERR_INVALID_ARG;
+  if (d_k > sdpa::F32_DMAX || d_v > sdpa::F32_DMAX) return SDPA_ERR_UNSUPPORTED;
+  if (batch == 0 || heads == 0 || n_q == 0) return SDPA_OK;
+  if (!Q || !K || !V || !O) return SDPA_ERR_INVALID_ARG;
+  if (!aligned4(Q) || !aligned4(K) || !aligned4(V) || !aligned4(O) || (LSE && !aligned4(LSE)))
+    return SDPA_ERR_MISALIGNED;
+  const long long bh = (long long)batch * heads;
+  if (bh > 65535 || bh * (long long)(n_q > n_kv ? n_q : n_kv) * 128 >= (1LL << 40)) return SDPA_ERR_UNSUPPORTED;
+  if (int e = check_device()) return e;
+  sdpa::F32Params p{Q, K, V, O, LSE, n_q, n_kv, d_k, d_v, scale, causal};
+  dim3 grid((unsigned)((n_q + sdpa::F32_ROWS - 1) / sdpa::F32_ROWS), (unsigned)bh);
+  sdpa::sdpa_fwd_f32_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+extern "C" size_t sdpa_decode_workspace_size(int batch, int heads, int n_kv_cap, int d_v) {
+  if (batch <= 0 || heads <= 0 || n_kv_cap <= 0 || d_v <= 0) return 0;
+  return decode_ws_bytes(batch, heads, n_kv_cap, d_v);
+}
+
+extern "C" int sdpa_decode(const void* Q, const void* K, const void* V, const int* kv_lens, void* O,
+                           float* LSE, int batch, int heads, int n_kv_cap, int d_k, int d_v, float scale,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (batch < 0 || heads < 0 || n_kv_cap < 1 || !std::isfinite(scale)) return SDPA_ERR_INVALID_ARG;
+  if (d_k != d_v || (d_k != 64 && d_k != 128)) return SDPA_ERR_UNSUPPORTED;
+  if (batch == 0 || heads == 0) return SDPA_OK;
+  if (!Q || !K || !V || !kv_lens || !O) return SDPA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned4(kv_lens) ||
+      (LSE && !aligned4(LSE)))
+    return SDPA_ERR_MISALIGNED;
+  if (batch > 65535 || heads > 65535) return SDPA_ERR_UNSUPPORTED;
+  const size_t need = decode_ws_bytes(batch, heads, n_kv_cap, d_v);
+  if (!workspace || workspace_bytes < need) return SDPA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SDPA_ERR_MISALIGNED;
+  if (int e = check_device()) return e;
+  sdpa::DecodeParams p;
+  p.Q = (const __nv_bfloat16*)Q;
+  p.K = (const __nv_bfloat16*)K;
+  p.V = (const __nv_bfloat16*)V;
+  p.kv_lens = kv_lens;
+  p.H = heads;
+  p.n_cap = n_kv_cap;
+  p.chunk = sdpa::decode_chunk(batch, heads, n_kv_cap);
+  p.n_split = (n_kv_cap + p.chunk - 1) / p.chunk;
+  p.part_o = (float*)workspace;
+  p.part_lse = p.part_o + (size_t)batch * heads * p.n_split * d_v;
+  p.O = (__nv_bfloat16*)O;
+  p.LSE = LSE;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = (cudaStream_t)stream;
+  dim3 grid((unsigned)p.n_split, (unsigned)heads, (unsigned)batch);
+  if (d_k == 64) {
+    sdpa::sdpa_decode_split_kernel<64><<<grid, sdpa::DECODE_THREADS, 0, s>>>(p);
+    sdpa::sdpa_decode_combine_kernel<64><<<(unsigned)(batch * heads), 64, 0, s>>>(p);
+  } else {
+    sdpa::sdpa_decode_split_kernel<128><<<grid, sdpa::DECODE_THREADS, 0, s>>>(p);
+    sdpa::sdpa_decode_combine_kernel<128><<<(unsigned)(batch * heads), 128, 0, s>>>(p);
+  }
+  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+extern "C" int sdpa_get_last_device_error(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SDPA_ERR_CUDA;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, sdpa::g_sdpa_error, sizeof v) != cudaSuccess) return SDPA_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(sdpa::g_sdpa_error, &zero, sizeof zero) != cudaSuccess) return SDPA_ERR_CUDA;
+  return v;
+}
+
+extern "C" const char* sdpa_status_string(int status) {
+  switch (status) {
+    case SDPA_OK: return "SDPA_OK";
+    case SDPA_ERR_INVALID_ARG: return "SDPA_ERR_INVALID_ARG";
+    case SDPA_ERR_UNSUPPORTED: return "SDPA_ERR_UNSUPPORTED";
+    case SDPA_ERR_MISALIGNED: return "SDPA_ERR_MISALIGNED";
+    case SDPA_ERR_WORKSPACE: return "SDPA_ERR_WORKSPACE";
+    case SDPA_ERR_CUDA: return "SDPA_ERR_CUDA";
+    case SDPA_ERR_DEVICE_TIMEOUT: return "SDPA_ERR_DEVICE_TIMEOUT";
+    case SDPA_ERR_DEVICE_BAD_LENGTH: return "SDPA_ERR_DEVICE_BAD_LENGTH";
+    default: return "SDPA_UNKNOWN_STATUS";
+  }
+}

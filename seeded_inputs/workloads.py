@@ -1,0 +1,122 @@
+"""The five synthetic workloads and their seeded inputs (shapes and value distributions only).
+
+  cfg1  fp32 prefill, B=1 H=1 n_q=n_kv=128 d=64, Q,K,V ~ N(0,1), scale 1/8, non-causal
+  cfg2  bf16 prefill, B=4 H=16 n=2048 d=64, Q,K,V ~ N(0,1), scale 1/8, non-causal and causal
+  cfg3  bf16 prefill, B=1 H=32 n=8192 d=128, Q,K ~ N(0,1), V ~ U(-1,1), scale 1/sqrt(128), causal
+  cfg4  bf16 prefill, B=1 H=8 n=32768 d=128, Q,K ~ N(0, 2.5^2), V ~ N(0,1), scale 1/sqrt(128), non-causal
+  cfg5  bf16 decode, B=64 H=32 n_cap=16384 d=128, lengths ~ U{1024..16384}, N(0,1), scale 1/sqrt(128)
+
+Streams: Q = 0, K = 1, V = 2 (counter = flat element index of the tensor), decode
+lengths = 3, sampled rows = 4.  Seed 0 everywhere.  bf16 values are the RNE
+rounding of the float32 draw; both the oracle and the GPU consume those bits.
+"""
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from . import NORMAL, UNIFORM, STREAM_Q, STREAM_K, STREAM_V, bf16_bits_to_f32, fill_host, kv_lengths
+
+
+@dataclass(frozen=True)
+class Dist:
+    kind: int = NORMAL
+    a: float = 0.0  # mean (normal) or low (uniform)
+    b: float = 1.0  # std (normal) or high (uniform)
+
+
+@dataclass(frozen=True)
+class Prefill:
+    name: str
+    batch: int
+    heads: int
+    n_q: int
+    n_kv: int
+    d: int
+    causal: bool
+    dtype: str  # "bf16" or "f32"
+    scale: float
+    q: Dist = field(default_factory=Dist)
+    k: Dist = field(default_factory=Dist)
+    v: Dist = field(default_factory=Dist)
+    seed: int = 0
+
+    @property
+    def scale_f32(self):
+        return float(np.float32(self.scale))
+
+    def flops(self):
+        """Algorithmic FLOPs: two matmuls at 2 FLOP per multiply-add, halved under a causal mask."""
+        f = 2.0 * self.batch * self.heads * self.n_q * self.n_kv * (2 * self.d)
+        return f / 2 if self.causal else f
+
+    def bytes(self):
+        """Algorithmic bytes: Q, K, V read and O, LSE written once."""
+        el = 2 if self.dtype == "bf16" else 4
+        bh = self.batch * self.heads
+        return bh * (self.n_q * self.d * 2 + self.n_kv * self.d * 2) * el + bh * self.n_q * 4
+
+    def with_causal(self, causal):
+        return Prefill(**{**self.__dict__, "causal": causal, "name": self.name + ("c" if causal else "")})
+
+
+@dataclass(frozen=True)
+class Decode:
+    name: str
+    batch: int
+    heads: int
+    n_cap: int
+    d: int
+    len_lo: int
+    len_hi: int
+    scale: float
+    seed: int = 0
+
+    @property
+    def scale_f32(self):
+        return float(np.float32(self.scale))
+
+    def lengths(self):
+        return kv_lengths(self.batch, self.len_lo, self.len_hi, self.seed)
+
+    def bytes(self, lens=None):
+        """Algorithmic bytes: the valid K and V rows, Q, O and LSE (bf16 except LSE)."""
+        lens = self.lengths() if lens is None else lens
+        kv = int(np.sum(lens, dtype=np.int64)) * self.heads * self.d * 2 * 2
+        return kv + self.batch * self.heads * (self.d * 2 * 2 + 4)
+
+    def flops(self, lens=None):
+        """Per token n(2 d_K + 2 d_V + 3) (standard attention's decode cost)."""
+        lens = self.lengths() if lens is None else lens
+        return float(np.sum(lens, dtype=np.int64)) * self.heads * (4 * self.d + 3)
+
+
+CFG1 = Prefill("cfg1", 1, 1, 128, 128, 64, False, "f32", 1 / 8)
+CFG2 = Prefill("cfg2", 4, 16, 2048, 2048, 64, False, "bf16", 1 / 8)
+CFG2C = CFG2.with_causal(True)
+CFG3 = Prefill("cfg3", 1, 32, 8192, 8192, 128, True, "bf16", 1 / 128 ** 0.5, v=Dist(UNIFORM, -1.0, 1.0))
+CFG4 = Prefill("cfg4", 1, 8, 32768, 32768, 128, False, "bf16", 1 / 128 ** 0.5, q=Dist(NORMAL, 0.0, 2.5),
+               k=Dist(NORMAL, 0.0, 2.5))
+CFG5 = Decode("cfg5", 64, 32, 16384, 128, 1024, 16384, 1 / 128 ** 0.5)
+
+
+def prefill_host(w):
+    """Host inputs of a prefill workload: dict of arrays; bf16 as uint16 bits, f32 as float32."""
+    bf = w.dtype == "bf16"
+    out = {}
+    for name, stream, dist, n in (("q", STREAM_Q, w.q, w.n_q), ("k", STREAM_K, w.k, w.n_kv),
+                                  ("v", STREAM_V, w.v, w.n_kv)):
+        out[name] = fill_host((w.batch, w.heads, n, w.d), w.seed, stream, dist.kind, dist.a, dist.b, bf16=bf)
+    return out
+
+
+def as_f32(x):
+    """Exact float32 view of host inputs (bf16 bits widen exactly)."""
+    return bf16_bits_to_f32(x) if x.dtype == np.uint16 else x
+
+
+def to_torch(x, device):
+    """Host array (uint16 bf16 bits or float32) -> torch tensor on `device`, same bits."""
+    import torch
+    if x.dtype == np.uint16:
+        return torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(x).to(device)

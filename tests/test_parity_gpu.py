@@ -1,0 +1,258 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded inputs.
+
+Tolerances: bf16 outputs |O - O_ref| <= 1e-2 + 1e-2 |O_ref| elementwise; fp32
+path |O - O_ref| <= 1e-5 |O_ref| + 1e-6; LSE within 1e-3 (natural-log units,
+absolute) for bf16 and 1e-5 for fp32; rows that see no key must give O = 0
+and LSE = -inf exactly.  Small cases compare every output against the oracle;
+the full-size workloads, run through the same call the benchmark times,
+compare seeded samples of query rows (or (batch, head) pairs for decode).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import seeded_inputs as si
+from seeded_inputs import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+BF16_ATOL, BF16_RTOL, LSE_TOL = 1e-2, 1e-2, 1e-3
+
+
+@pytest.fixture(scope="module")
+def sdpa(cuda_device):
+    import memory_optimal_sdpa_b200 as m
+    return m
+
+
+def _bits_to_torch(bits, device, pad_nan=0):
+    """bf16 bits -> CUDA bf16 tensor, placed at the start of a buffer whose `pad_nan` trailing elements are NaN."""
+    import torch
+    flat = torch.full((bits.size + pad_nan,), float("nan"), dtype=torch.bfloat16, device=device)
+    flat[:bits.size] = torch.from_numpy(bits.reshape(-1).view(np.int16)).to(device).view(torch.bfloat16)
+    return flat, flat[:bits.size].view(bits.shape)
+
+
+def _nan_buffer(shape, dtype, device, pad):
+    import torch
+    n = int(np.prod(shape))
+    flat = torch.full((n + pad,), float("nan"), dtype=dtype, device=device)
+    return flat, flat[:n].view(shape)
+
+
+def check_bf16(O, O_ref, L, L_ref, what):
+    O = O.astype(np.float64)
+    err = np.abs(O - O_ref)
+    bound = BF16_ATOL + BF16_RTOL * np.abs(O_ref)
+    bad = ~(err <= bound)
+    assert not bad.any(), "%s: %d/%d outputs out of bound, worst excess %.3g at %s" % (
+        what, bad.sum(), bad.size, np.nanmax(err - bound), np.unravel_index(np.argmax(np.where(bad, err - bound, -1)), bad.shape))
+    check_lse(L, L_ref, LSE_TOL, what)
+
+
+def check_lse(L, L_ref, tol, what):
+    L = L.astype(np.float64)
+    masked = np.isneginf(L_ref)
+    assert (np.isneginf(L) == masked).all(), what + ": -inf LSE pattern differs"
+    d = np.abs(L[~masked] - L_ref[~masked])
+    assert (d <= tol).all(), "%s: LSE max err %.3g" % (what, d.max())
+
+
+# ----------------------------------------------------------------------------- bf16 prefill, small, every row
+SMALL = [
+    # (batch, heads, n_q, n_kv, d, causal)
+    (1, 2, 128, 128, 64, False), (1, 2, 128, 128, 64, True),
+    (1, 2, 128, 128, 128, False), (1, 2, 128, 128, 128, True),
+    (2, 3, 257, 257, 64, True), (1, 3, 1000, 1000, 128, True), (1, 3, 1000, 1000, 64, False),
+    (1, 2, 1, 1, 64, False), (1, 2, 1, 1, 128, True), (1, 2, 2, 129, 128, True), (1, 3, 127, 255, 64, True),
+    (1, 2, 255, 2, 64, False), (1, 2, 300, 100, 128, True), (1, 1, 129, 1, 64, False),
+    (2, 2, 512, 384, 128, False), (1, 3, 600, 1000, 64, True), (1, 1, 513, 777, 128, True),
+    (3, 1, 256, 512, 64, False),
+]
+
+
+@pytest.mark.parametrize("B,H,n_q,n_kv,d,causal", SMALL)
+def test_prefill_bf16_small(sdpa, cuda_device, B, H, n_q, n_kv, d, causal):
+    import torch
+    seed = hash((B, H, n_q, n_kv, d, causal)) & 0xFFFF
+    q = si.fill_host((B, H, n_q, d), seed, 0)
+    k = si.fill_host((B, H, n_kv, d), seed, 1)
+    v = si.fill_host((B, H, n_kv, d), seed, 2)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    pad = 128 * d
+    _, tq = _bits_to_torch(q, cuda_device, pad)
+    _, tk = _bits_to_torch(k, cuda_device, pad)
+    _, tv = _bits_to_torch(v, cuda_device, pad)
+    o_flat, o = _nan_buffer((B, H, n_q, d), torch.bfloat16, cuda_device, pad)
+    l_flat, lse = _nan_buffer((B, H, n_q), torch.float32, cuda_device, 256)
+    sdpa.fwd(tq, tk, tv, causal=causal, scale=scale, o=o, lse=lse)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O_ref, L_ref = oracle.sdpa_rows(si.bf16_bits_to_f32(q), si.bf16_bits_to_f32(k), si.bf16_bits_to_f32(v), scale, causal)
+    check_bf16(o.float().cpu().numpy(), O_ref, lse.cpu().numpy(), L_ref, "prefill %s" % ((B, H, n_q, n_kv, d, causal),))
+    # guard bands after the outputs are untouched
+    assert torch.isnan(o_flat[o.numel():]).all() and torch.isnan(l_flat[lse.numel():]).all()
+    # fully masked rows (causal, n_q > n_kv): exactly zero output
+    if causal and n_q > n_kv:
+        O = o.float().cpu().numpy()
+        assert (O[:, :, :n_q - n_kv] == 0).all()
+
+
+def test_prefill_lse_optional_and_repeatable(sdpa, cuda_device):
+    import torch
+    B, H, n, d = 1, 4, 384, 128
+    q, k, v = (W.to_torch(si.fill_host((B, H, n, d), 7, s), cuda_device) for s in (0, 1, 2))
+    o1, l1 = sdpa.fwd(q, k, v, causal=True)
+    o2, _ = sdpa.fwd(q, k, v, causal=True, want_lse=False)
+    o3, l3 = sdpa.fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(o1, o3) and torch.equal(l1, l3)
+
+
+def test_prefill_shift_invariance_on_gpu(sdpa, cuda_device):
+    # K' = K + 1 u^T adds scale*(q_i . u) to row i's logits: O unchanged, LSE shifted (exact in bf16 for small ints)
+    import torch
+    B, H, n, d = 1, 2, 256, 64
+    g = np.random.default_rng(3)
+    qf = g.integers(-2, 3, (B, H, n, d)).astype(np.float32)
+    kf = g.integers(-2, 3, (B, H, n, d)).astype(np.float32)
+    u = g.integers(-2, 3, (d,)).astype(np.float32)
+    vf = si.bf16_bits_to_f32(si.fill_host((B, H, n, d), 1, 2))
+    to = lambda a: torch.from_numpy(a).to(cuda_device).to(torch.bfloat16)
+    o1, l1 = sdpa.fwd(to(qf), to(kf), to(vf), scale=0.125)
+    o2, l2 = sdpa.fwd(to(qf), to(kf + u), to(vf), scale=0.125)
+    shift = 0.125 * np.einsum("bhnd,d->bhn", qf.astype(np.float64), u.astype(np.float64))
+    np.testing.assert_allclose(o2.float().cpu().numpy(), o1.float().cpu().numpy(), atol=2e-2, rtol=2e-2)
+    np.testing.assert_allclose(l2.cpu().numpy(), l1.cpu().numpy() + shift, atol=2e-3, rtol=0)
+
+
+# ------------------------------------------------------------------ bf16 prefill, full-size workloads, sampled rows
+def _sampled_prefill(sdpa, device, w, rows_per_head):
+    import torch
+    host = W.prefill_host(w)
+    tq, tk, tv = (W.to_torch(host[n], device) for n in ("q", "k", "v"))
+    o, lse = sdpa.fwd(tq, tk, tv, causal=w.causal, scale=w.scale_f32)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O = o.float().cpu().numpy()
+    L = lse.cpu().numpy()
+    del tq, tk, tv, o, lse
+    torch.cuda.empty_cache()
+    qf, kf, vf = (W.as_f32(host[n]) for n in ("q", "k", "v"))
+    for b in range(w.batch):
+        for h in range(w.heads):
+            rows = si.sample_rows(w.n_q, rows_per_head, w.seed, salt=b * w.heads + h)
+            O_ref, L_ref = oracle.sdpa_rows(qf[b, h], kf[b, h], vf[b, h], w.scale_f32, w.causal, rows=rows)
+            check_bf16(O[b, h, rows], O_ref, L[b, h, rows], L_ref, "%s b=%d h=%d" % (w.name, b, h))
+
+
+def test_cfg2_noncausal_sampled(sdpa, cuda_device):
+    _sampled_prefill(sdpa, cuda_device, W.CFG2, 64)
+
+
+def test_cfg2_causal_sampled(sdpa, cuda_device):
+    _sampled_prefill(sdpa, cuda_device, W.CFG2C, 64)
+
+
+def test_cfg3_causal_sampled(sdpa, cuda_device):
+    _sampled_prefill(sdpa, cuda_device, W.CFG3, 256)
+
+
+def test_cfg4_long_sampled(sdpa, cuda_device):
+    _sampled_prefill(sdpa, cuda_device, W.CFG4, 256)
+
+
+# ----------------------------------------------------------------------------------------------- fp32 path
+F32_CASES = [(1, 1, 128, 128, 64, 64, False), (1, 1, 128, 128, 64, 64, True), (2, 3, 77, 130, 33, 100, True),
+             (1, 2, 200, 50, 128, 128, True), (1, 1, 1, 1, 1, 1, False), (1, 2, 65, 300, 3, 128, False)]
+
+
+@pytest.mark.parametrize("B,H,n_q,n_kv,dk,dv,causal", F32_CASES)
+def test_prefill_f32(sdpa, cuda_device, B, H, n_q, n_kv, dk, dv, causal):
+    q = si.fill_host((B, H, n_q, dk), 0, 0, bf16=False)
+    k = si.fill_host((B, H, n_kv, dk), 0, 1, bf16=False)
+    v = si.fill_host((B, H, n_kv, dv), 0, 2, bf16=False)
+    scale = float(np.float32(1 / math.sqrt(dk)))
+    tq, tk, tv = (W.to_torch(x, cuda_device) for x in (q, k, v))
+    o, lse = sdpa.fwd_f32(tq, tk, tv, causal=causal, scale=scale)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O_ref, L_ref = oracle.sdpa_rows(q, k, v, scale, causal)
+    O = o.cpu().numpy().astype(np.float64)
+    err = np.abs(O - O_ref)
+    assert (err <= 1e-5 * np.abs(O_ref) + 1e-6).all(), "max rel err %.3g" % (err / (np.abs(O_ref) + 1e-6)).max()
+    check_lse(lse.cpu().numpy(), L_ref, 1e-5, "f32")
+
+
+def test_cfg1_fp32(sdpa, cuda_device):
+    w = W.CFG1
+    host = W.prefill_host(w)
+    tq, tk, tv = (W.to_torch(host[n], cuda_device) for n in ("q", "k", "v"))
+    o, lse = sdpa.fwd_f32(tq, tk, tv, causal=w.causal, scale=w.scale_f32)
+    O_ref, L_ref = oracle.sdpa_rows(host["q"], host["k"], host["v"], w.scale_f32, w.causal)
+    O = o.cpu().numpy().astype(np.float64)
+    assert (np.abs(O - O_ref) <= 1e-5 * np.abs(O_ref) + 1e-6).all()
+    check_lse(lse.cpu().numpy(), L_ref, 1e-5, "cfg1")
+
+
+# -------------------------------------------------------------------------------------------------- decode
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_small_every_pair(sdpa, cuda_device, d):
+    import torch
+    B, H, n_cap = 3, 4, 1000
+    lens = np.array([1, 1000, 517], np.int32)
+    q = si.fill_host((B, H, d), 5, 0)
+    k = si.fill_host((B, H, n_cap, d), 5, 1)
+    v = si.fill_host((B, H, n_cap, d), 5, 2)
+    for b in range(B):  # rows past the length hold NaN: any read of them poisons O
+        k[b, :, lens[b]:] = 0x7FC0
+        v[b, :, lens[b]:] = 0x7FC0
+    scale = float(np.float32(1 / math.sqrt(d)))
+    tq, tk, tv = (W.to_torch(x, cuda_device) for x in (q, k, v))
+    tl = torch.from_numpy(lens).to(cuda_device)
+    o, lse = sdpa.decode(tq, tk, tv, tl, scale=scale)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O_ref, L_ref = oracle.decode(si.bf16_bits_to_f32(q), si.bf16_bits_to_f32(k), si.bf16_bits_to_f32(v), lens, scale)
+    check_bf16(o.float().cpu().numpy().reshape(B * H, d), O_ref, lse.cpu().numpy().reshape(-1), L_ref, "decode d=%d" % d)
+
+
+def test_decode_bad_length_reported(sdpa, cuda_device):
+    import torch
+    B, H, n_cap, d = 2, 2, 64, 64
+    tq = torch.zeros((B, H, d), dtype=torch.bfloat16, device=cuda_device)
+    tk = torch.zeros((B, H, n_cap, d), dtype=torch.bfloat16, device=cuda_device)
+    tl = torch.tensor([5, 65], dtype=torch.int32, device=cuda_device)
+    sdpa.decode(tq, tk, tk, tl)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_ERR_DEVICE_BAD_LENGTH
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK  # read clears the word
+
+
+def test_cfg5_decode_full_size_sampled(sdpa, cuda_device):
+    import torch
+    w = W.CFG5
+    lens = w.lengths()
+    tl = torch.from_numpy(lens).to(cuda_device)
+    shape = (w.batch, w.heads, w.n_cap, w.d)
+    tk = torch.empty(shape, dtype=torch.bfloat16, device=cuda_device)
+    tv = torch.empty(shape, dtype=torch.bfloat16, device=cuda_device)
+    si.fill_device_cache(tk, tl, w.seed, si.STREAM_K)
+    si.fill_device_cache(tv, tl, w.seed, si.STREAM_V)
+    q = si.fill_host((w.batch, w.heads, w.d), w.seed, si.STREAM_Q)
+    o, lse = sdpa.decode(W.to_torch(q, cuda_device), tk, tv, tl, scale=w.scale_f32)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O = o.float().cpu().numpy().reshape(-1, w.d)
+    L = lse.cpu().numpy().reshape(-1)
+    del tk, tv
+    torch.cuda.empty_cache()
+    # pairs: both heads 0 and H-1 of the shortest and the longest sequence, plus seeded picks
+    b_min, b_max = int(np.argmin(lens)), int(np.argmax(lens))
+    picks = {b_min * w.heads, b_min * w.heads + w.heads - 1, b_max * w.heads, b_max * w.heads + w.heads - 1}
+    picks |= set(int(x) for x in si.sample_rows(w.batch * w.heads, 60, w.seed, salt=99))
+    qf = si.bf16_bits_to_f32(q).reshape(-1, w.d)
+    for bh in sorted(picks):
+        b, h = divmod(bh, w.heads)
+        n = int(lens[b])
+        start = ((b * w.heads + h) * w.n_cap) * w.d
+        kf = si.bf16_bits_to_f32(si.fill_host((n, w.d), w.seed, si.STREAM_K, start=start))
+        vf = si.bf16_bits_to_f32(si.fill_host((n, w.d), w.seed, si.STREAM_V, start=start))
+        O_ref, L_ref = oracle.sdpa_rows(qf[bh][None], kf, vf, w.scale_f32)
+        check_bf16(O[bh][None], O_ref, L[bh:bh + 1], L_ref, "cfg5 b=%d h=%d len=%d" % (b, h, n))
