@@ -9,11 +9,17 @@
 // 128-row tiles: one work unit is one (batch, head) and two adjacent 128-row
 // query tiles (a, b), streamed against 128-row key/value tiles.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax warpgroup for query tile a (thread t owns TMEM lane = row t)
 //   warps 4-7  softmax warpgroup for query tile b
 //   warp  8    TMA producer: Q once, then K_j, V_j into a ring of shared-memory slots
 //   warp  9    MMA issuer (one thread) and TMEM owner
+//   warps 10-11 idle
+// Registers: each SM sub-partition holds 16K 32-bit registers and receives
+// one warp of every warpgroup, so the CTA launches at 168 per thread and then
+// moves registers from the producer/MMA warpgroup (down to 56) to the two
+// softmax warpgroups (up to 224): 2*224 + 56 <= 512 per sub-partition lane
+// slot, and 56*128 + 224*256 = 384*168 in total.
 // TMEM (512 columns): S_a [0,128), S_b [128,256), O_a [256,256+D), O_b [384,384+D).
 // P_x (bf16, two per column) overwrites the first 64 columns of S_x once the
 // softmax has read S_x; the next S_x MMA is issued after the P_x V MMA, and
@@ -45,7 +51,9 @@ struct PrefillCfg {
   static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
   static constexpr int NBAR = 1 + 2 * NSLOT + 2 + 2 + 2 + 1;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;  // + tmem slot, abort flag, align slack
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;
+  static constexpr int SOFTMAX_REGS = 224;
+  static constexpr int CONTROL_REGS = 56;
   static constexpr int LOAD_WARP = 8;
   static constexpr int MMA_WARP = 9;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -75,7 +83,7 @@ struct PrefillParams {
 };
 
 template <int D, bool CAUSAL>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(384, 1)
     sdpa_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using C = PrefillCfg<D>;
@@ -130,108 +138,112 @@ __global__ void __maxnreg__(200)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   bool timed_out = false;
+  static_assert(C::SOFTMAX_REGS * 256 + C::CONTROL_REGS * 128 <= 168 * 384, "register split exceeds the launch");
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONTROL_REGS));
+    if (warp == C::LOAD_WARP) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0 && T > 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
+  #pragma unroll
+        for (int x = 0; x < 2; ++x)
+  #pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_3d(sQ + x * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmQ, q_full, cb * 64, x ? r0b : r0a, bh);
+        int issued = 0;
+        for (int idx = 0; idx < 2 * T; ++idx) {
+          const int slot = idx % C::NSLOT;
+          const uint32_t ph = (uint32_t)(idx / C::NSLOT) & 1u;
+          if (!mbar_wait_bounded(&empty[slot], ph ^ 1u, abort_flag, &timed_out)) break;
+          mbar_arrive_expect_tx(&full[slot], C::TILE_BYTES);
+          const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
+          uint8_t* dst = sKV + slot * C::TILE_BYTES;
+  #pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_3d(dst + cb * C::BLOCK_BYTES, map, &full[slot], cb * 64, (idx >> 1) * 128, bh);
+          issued = idx + 1;
+        }
+        if (*abort_flag) {  // let the copies already in flight land before the CTA exits
+          mbar_wait_drain(q_full, 0);
+          for (int idx = (issued > C::NSLOT ? issued - C::NSLOT : 0); idx < issued; ++idx)
+            mbar_wait_drain(&full[idx % C::NSLOT], (uint32_t)(idx / C::NSLOT) & 1u);
+        }
+      }
+    } else if (warp == C::MMA_WARP) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0 && T > 0) {
+        const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+        const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
+        constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
+        constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // P (TMEM) x V (MN-major)
+        const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
 
-  if (warp == C::LOAD_WARP) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && T > 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
-#pragma unroll
-      for (int x = 0; x < 2; ++x)
-#pragma unroll
-        for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_3d(sQ + x * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmQ, q_full, cb * 64, x ? r0b : r0a, bh);
-      int issued = 0;
-      for (int idx = 0; idx < 2 * T; ++idx) {
-        const int slot = idx % C::NSLOT;
-        const uint32_t ph = (uint32_t)(idx / C::NSLOT) & 1u;
-        if (!mbar_wait_bounded(&empty[slot], ph ^ 1u, abort_flag, &timed_out)) break;
-        mbar_arrive_expect_tx(&full[slot], C::TILE_BYTES);
-        const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
-        uint8_t* dst = sKV + slot * C::TILE_BYTES;
-#pragma unroll
-        for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_3d(dst + cb * C::BLOCK_BYTES, map, &full[slot], cb * 64, (idx >> 1) * 128, bh);
-        issued = idx + 1;
-      }
-      if (*abort_flag) {  // let the copies already in flight land before the CTA exits
-        mbar_wait_drain(q_full, 0);
-        for (int idx = (issued > C::NSLOT ? issued - C::NSLOT : 0); idx < issued; ++idx)
-          mbar_wait_drain(&full[idx % C::NSLOT], (uint32_t)(idx / C::NSLOT) & 1u);
-      }
-    }
-  } else if (warp == C::MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && T > 0) {
-      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-      const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
-      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
-      constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // P (TMEM) x V (MN-major)
-      const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
+        auto issue_S = [&](int x, int j) {  // S_x = Q_x K_j^T
+          const uint32_t qa = sQa + x * C::TILE_BYTES;
+          const uint32_t ka = sKVa + ((2 * j) % C::NSLOT) * C::TILE_BYTES;
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BLOCK_BYTES + (kk & 3) * 32;
+            mma_ss(tS[x], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), idS,
+                   kk > 0 ? 1u : 0u);
+          }
+        };
+        auto issue_PV = [&](int x, int j) {  // O_x += P_x V_j
+          const uint32_t va = sKVa + ((2 * j + 1) % C::NSLOT) * C::TILE_BYTES;
+  #pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            mma_ts(tO[x], tS[x] + kk * 8, smem_desc_sw128(va + kk * 2048, C::BLOCK_BYTES, 1024), idO,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+        };
+        auto wait_slot = [&](int idx) {
+          return mbar_wait_bounded(&full[idx % C::NSLOT], (uint32_t)(idx / C::NSLOT) & 1u, abort_flag,
+                                   &timed_out);
+        };
 
-      auto issue_S = [&](int x, int j) {  // S_x = Q_x K_j^T
-        const uint32_t qa = sQa + x * C::TILE_BYTES;
-        const uint32_t ka = sKVa + ((2 * j) % C::NSLOT) * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BLOCK_BYTES + (kk & 3) * 32;
-          mma_ss(tS[x], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), idS,
-                 kk > 0 ? 1u : 0u);
+        bool ok = mbar_wait_bounded(q_full, 0, abort_flag, &timed_out) && wait_slot(0);
+        if (ok) {
+          tc_fence_after_sync();
+          if (ta > 0) { issue_S(0, 0); tc_commit(&s_full[0]); }
+          if (tb > 0) { issue_S(1, 0); tc_commit(&s_full[1]); }
+          tc_commit(&empty[0]);
         }
-      };
-      auto issue_PV = [&](int x, int j) {  // O_x += P_x V_j
-        const uint32_t va = sKVa + ((2 * j + 1) % C::NSLOT) * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tO[x], tS[x] + kk * 8, smem_desc_sw128(va + kk * 2048, C::BLOCK_BYTES, 1024), idO,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-      };
-      auto wait_slot = [&](int idx) {
-        return mbar_wait_bounded(&full[idx % C::NSLOT], (uint32_t)(idx / C::NSLOT) & 1u, abort_flag,
-                                 &timed_out);
-      };
-
-      bool ok = mbar_wait_bounded(q_full, 0, abort_flag, &timed_out) && wait_slot(0);
-      if (ok) {
-        tc_fence_after_sync();
-        if (ta > 0) { issue_S(0, 0); tc_commit(&s_full[0]); }
-        if (tb > 0) { issue_S(1, 0); tc_commit(&s_full[1]); }
-        tc_commit(&empty[0]);
+        for (int j = 0; ok && j < T; ++j) {
+          if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
+          tc_fence_after_sync();
+          if (j < ta) {
+            if (!(ok = mbar_wait_bounded(&p_full[0], (uint32_t)j & 1u, abort_flag, &timed_out))) break;
+            tc_fence_after_sync();
+            issue_PV(0, j);
+            if (j == ta - 1) tc_commit(&o_full[0]);
+          }
+          if (j + 1 < T) {
+            if (!(ok = wait_slot(2 * (j + 1)))) break;  // K_{j+1}
+            tc_fence_after_sync();
+            if (j + 1 < ta) { issue_S(0, j + 1); tc_commit(&s_full[0]); }
+          }
+          if (j < tb) {
+            if (!(ok = mbar_wait_bounded(&p_full[1], (uint32_t)j & 1u, abort_flag, &timed_out))) break;
+            tc_fence_after_sync();
+            issue_PV(1, j);
+            if (j == tb - 1) tc_commit(&o_full[1]);
+          }
+          tc_commit(&empty[(2 * j + 1) % C::NSLOT]);  // V_j slot free once both PV MMAs are done
+          if (j + 1 < T) {
+            if (j + 1 < tb) { issue_S(1, j + 1); tc_commit(&s_full[1]); }
+            tc_commit(&empty[(2 * (j + 1)) % C::NSLOT]);  // K_{j+1} slot
+          }
+        }
+        // Every MMA and every commit issued above has landed before TMEM is released
+        // and before the CTA's shared memory (which the commits arrive on) goes away.
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0);
       }
-      for (int j = 0; ok && j < T; ++j) {
-        if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
-        tc_fence_after_sync();
-        if (j < ta) {
-          if (!(ok = mbar_wait_bounded(&p_full[0], (uint32_t)j & 1u, abort_flag, &timed_out))) break;
-          tc_fence_after_sync();
-          issue_PV(0, j);
-          if (j == ta - 1) tc_commit(&o_full[0]);
-        }
-        if (j + 1 < T) {
-          if (!(ok = wait_slot(2 * (j + 1)))) break;  // K_{j+1}
-          tc_fence_after_sync();
-          if (j + 1 < ta) { issue_S(0, j + 1); tc_commit(&s_full[0]); }
-        }
-        if (j < tb) {
-          if (!(ok = mbar_wait_bounded(&p_full[1], (uint32_t)j & 1u, abort_flag, &timed_out))) break;
-          tc_fence_after_sync();
-          issue_PV(1, j);
-          if (j == tb - 1) tc_commit(&o_full[1]);
-        }
-        tc_commit(&empty[(2 * j + 1) % C::NSLOT]);  // V_j slot free once both PV MMAs are done
-        if (j + 1 < T) {
-          if (j + 1 < tb) { issue_S(1, j + 1); tc_commit(&s_full[1]); }
-          tc_commit(&empty[(2 * (j + 1)) % C::NSLOT]);  // K_{j+1} slot
-        }
-      }
-      // Every MMA and every commit issued above has landed before TMEM is released
-      // and before the CTA's shared memory (which the commits arrive on) goes away.
-      tc_commit(drain);
-      mbar_wait_drain(drain, 0);
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
     // ------------------------------------------------ softmax + epilogue warpgroups
     const int x = warp >> 2;  // query tile a (0) or b (1)
     const int t = threadIdx.x & 127;

@@ -6,6 +6,8 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "sdpa.h"
@@ -14,6 +16,19 @@
 #include "decode.cuh"
 
 namespace {
+
+// SDPA_DEBUG=1 in the environment: report the failing CUDA call on stderr.
+bool debug_on() {
+  static const bool on = [] {
+    const char* e = std::getenv("SDPA_DEBUG");
+    return e && e[0] && e[0] != '0';
+  }();
+  return on;
+}
+int cuda_fail(const char* what, cudaError_t e) {
+  if (debug_on()) std::fprintf(stderr, "sdpa: %s failed: %s\n", what, cudaGetErrorString(e));
+  return SDPA_ERR_CUDA;
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
@@ -26,9 +41,12 @@ EncodeTiledFn encode_fn() {
   std::call_once(once, [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e == cudaSuccess && q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<EncodeTiledFn>(p);
+    else if (debug_on())
+      std::fprintf(stderr, "sdpa: cuTensorMapEncodeTiled entry point not found (%s, query %d)\n",
+                   cudaGetErrorString(e), (int)q);
   });
   return fn;
 }
@@ -41,9 +59,12 @@ bool make_map(CUtensorMap* map, const void* ptr, int d, int n, int bh) {
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && debug_on())
+    std::fprintf(stderr, "sdpa: cuTensorMapEncodeTiled failed (CUresult %d) d=%d n=%d bh=%d\n", (int)r, d, n, bh);
+  return r == CUDA_SUCCESS;
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -71,7 +92,7 @@ int launch_prefill(const void* Q, const void* K, const void* V, void* O, float* 
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   });
-  if (attr_err != cudaSuccess) return SDPA_ERR_CUDA;
+  if (attr_err != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem)", attr_err);
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, Q, D, n_q, bh) || !make_map(&mk, K, D, n_kv, bh) || !make_map(&mv, V, D, n_kv, bh))
     return SDPA_ERR_CUDA;
@@ -85,7 +106,17 @@ int launch_prefill(const void* Q, const void* K, const void* V, void* O, float* 
   p.scale_log2 = scale * 1.4426950408889634f;
   const long long grid = (long long)bh * p.n_pairs;
   kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess && debug_on()) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess)
+      std::fprintf(stderr,
+                   "sdpa: prefill<%d,%d> regs %d maxThreads %d static smem %zu max dyn smem %d local %zu; "
+                   "launch %lld x %d threads, %d B dynamic smem\n",
+                   D, (int)CAUSAL, fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes,
+                   fa.maxDynamicSharedSizeBytes, fa.localSizeBytes, grid, Cfg::THREADS, Cfg::SMEM_BYTES);
+  }
+  return e == cudaSuccess ? SDPA_OK : cuda_fail("prefill launch", e);
 }
 
 size_t decode_ws_bytes(long long batch, long long heads, long long n_cap, long long d_v) {
