@@ -1,0 +1,74 @@
+"""Host-side logic of bench.py: cross-rank aggregation over gloo (2 ranks, CPU) and the JSON helpers."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    import datetime
+    import torch.distributed as dist
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    # rank r timed (r+1) seconds for 10*(r+1) units of work
+    t, u = bench.aggregate(float(rank + 1), 10.0 * (rank + 1))
+    bench.barrier()
+    out[rank] = (t, u)
+    dist.destroy_process_group()
+
+
+def test_aggregate_max_time_sum_units_over_gloo():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    # every rank sees the slowest rank's time and the work of all ranks
+    assert res == {0: (2.0, 30.0), 1: (2.0, 30.0)}
+
+
+def test_aggregate_single_process_is_identity():
+    import bench
+    assert bench.aggregate(1.5, 7.0) == (1.5, 7.0)
+
+
+def test_reference_arm_rank_nonzero_does_nothing(capsys, monkeypatch):
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    assert capsys.readouterr().out == ""
+
+
+def test_warmup_floor():
+    import bench
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2"])
+
+
+def test_traffic_is_null_when_kernel_changed(tmp_path, monkeypatch):
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "k.cuh"
+    src.write_text("kernel v1")
+    digest = bench.source_digest(["k.cuh"])
+    (tmp_path / "profiles" / "p.txt").write_text("source_digest: %s\ndram_bytes_per_launch_full_workload: 123\n" % digest)
+    assert bench.profiled_traffic("p.txt", ["k.cuh"]) == 123.0
+    src.write_text("kernel v2")
+    assert bench.profiled_traffic("p.txt", ["k.cuh"]) is None
