@@ -114,6 +114,39 @@ SDPA_API int sdpa_decode(const void* Q, const void* K, const void* V, const int*
                 size_t workspace_bytes, void* stream);
 
 /*
+ * sdpa_decode_noalloc -- sdpa_decode for callers that cannot allocate device memory.
+ *
+ * The attention pages have no counterpart to this entry point; it exists for
+ * callers that are not allowed to call cudaMalloc or to hold a workspace
+ * buffer -- for example a plug-in whose host application owns every device
+ * allocation, or code running under a fixed memory budget where a framework's
+ * allocator is the only one permitted.  It computes exactly what sdpa_decode
+ * computes, with the same arguments minus the workspace, and allocates nothing:
+ * its scratch (the per-split partial outputs and log-sum-exps) lives in one
+ * library-owned device array of SDPA_DECODE_STATIC_SCRATCH_BYTES, which every
+ * GPU that loads this library holds until the process exits.
+ *
+ *  - Size limit: batch * heads * splits * (d_v + 1) * 4 bytes must fit in the array.
+ *    The call picks the smallest key-split length (a power of two, at least the
+ *    one sdpa_decode uses) that fits; if even one split per (batch, head) does not
+ *    fit (batch * heads * (d_v + 1) * 4 > SDPA_DECODE_STATIC_SCRATCH_BYTES) it
+ *    returns SDPA_ERR_WORKSPACE before launching anything.
+ *  - Set-up: the first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current.  Make that first call on
+ *    every device before any stream capture begins.
+ *  - Sharing: every call uses the same array and it keeps the last call's
+ *    contents.  Nothing in it needs to start at zero (each call writes every
+ *    partial it reads).  Calls whose work overlaps on the GPU (other streams,
+ *    other host threads on the same device) race on the array: serialise them.
+ *  - Results may differ from sdpa_decode in the last bits, because the key
+ *    splits can be longer.
+ */
+#define SDPA_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
+SDPA_API int sdpa_decode_noalloc(const void* Q, const void* K, const void* V, const int* kv_lens, void* O,
+                                 float* LSE, int batch, int heads, int n_kv_cap, int d_k, int d_v, float scale,
+                                 void* stream);
+
+/*
  * sdpa_get_last_device_error -- synchronise `stream`, then read and clear the
  * device error word of the current device.  Returns SDPA_OK, the first device
  * error recorded since the last call, or SDPA_ERR_CUDA if the synchronisation

@@ -31,6 +31,8 @@ lib.sdpa_decode_workspace_size.argtypes = [_i, _i, _i, _i]
 lib.sdpa_decode_workspace_size.restype = _sz
 lib.sdpa_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]
 lib.sdpa_decode.restype = _i
+lib.sdpa_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp]
+lib.sdpa_decode_noalloc.restype = _i
 lib.sdpa_get_last_device_error.argtypes = [_vp]
 lib.sdpa_get_last_device_error.restype = _i
 lib.sdpa_status_string.argtypes = [_i]
@@ -123,6 +125,25 @@ def decode(q, k, v, kv_lens, scale=None, o=None, lse=None, want_lse=True, worksp
     _check(lib.sdpa_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), _ptr(o), _ptr(lse), B, H, n_cap, d_k, d_v,
                            float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
                            _stream(stream)), "sdpa_decode")
+    return o, lse
+
+
+def decode_noalloc(q, k, v, kv_lens, scale=None, o=None, lse=None, want_lse=True, stream=None):
+    """Decode without a workspace: for callers that may not allocate device memory.
+
+    Uses the library's fixed device scratch array (see sdpa_decode_noalloc in
+    include/sdpa.h).  o and lse are allocated here only when not given.
+    """
+    import torch
+    B, H, n_cap, d_k = k.shape
+    d_v = v.shape[3]
+    scale = 1.0 / math.sqrt(d_k) if scale is None else scale
+    if o is None:
+        o = torch.empty((B, H, d_v), dtype=q.dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    _check(lib.sdpa_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), _ptr(o), _ptr(lse), B, H, n_cap, d_k,
+                                   d_v, float(scale), _stream(stream)), "sdpa_decode_noalloc")
     return o, lse
 
 

@@ -215,6 +215,95 @@ extern "C" int sdpa_decode(const void* Q, const void* K, const void* V, const in
   return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ sdpa_decode_noalloc
+// Scratch for callers that cannot allocate: one fixed array per device that loads
+// this library.  Host code must never pass `g_decode_static_scratch` itself to a
+// kernel (on the host it names a stand-in, not device memory); it passes the
+// address cudaGetSymbolAddress returns for the current device.
+namespace {
+constexpr size_t kStaticScratchFloats = SDPA_DECODE_STATIC_SCRATCH_BYTES / sizeof(float);
+__device__ __align__(256) float g_decode_static_scratch[kStaticScratchFloats];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_scratch_mutex;
+float* g_static_scratch_ptr[kMaxDevices];
+
+// Device address of the scratch array on the current device (looked up once per device).
+float* static_scratch_for_current_device(int* status) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    *status = cuda_fail("cudaGetDevice", e);
+    return nullptr;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {
+    *status = SDPA_ERR_UNSUPPORTED;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+  if (!g_static_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_static_scratch);
+    if (e != cudaSuccess || !p) {
+      *status = cuda_fail("cudaGetSymbolAddress(static decode scratch)", e);
+      return nullptr;
+    }
+    g_static_scratch_ptr[dev] = static_cast<float*>(p);
+  }
+  *status = SDPA_OK;
+  return g_static_scratch_ptr[dev];
+}
+}  // namespace
+
+extern "C" int sdpa_decode_noalloc(const void* Q, const void* K, const void* V, const int* kv_lens, void* O,
+                                   float* LSE, int batch, int heads, int n_kv_cap, int d_k, int d_v, float scale,
+                                   void* stream) {
+  if (batch < 0 || heads < 0 || n_kv_cap < 1 || !std::isfinite(scale)) return SDPA_ERR_INVALID_ARG;
+  if (d_k != d_v || (d_k != 64 && d_k != 128)) return SDPA_ERR_UNSUPPORTED;
+  if (batch == 0 || heads == 0) return SDPA_OK;
+  if (!Q || !K || !V || !kv_lens || !O) return SDPA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned4(kv_lens) ||
+      (LSE && !aligned4(LSE)))
+    return SDPA_ERR_MISALIGNED;
+  if (batch > 65535 || heads > 65535) return SDPA_ERR_UNSUPPORTED;
+  // Smallest split length (from the one sdpa_decode uses, doubling) whose partials fit the array.
+  const long long bh = (long long)batch * heads;
+  long long chunk = sdpa::decode_chunk(batch, heads, n_kv_cap);
+  while (bh * ((n_kv_cap + chunk - 1) / chunk) * (d_v + 1) > (long long)kStaticScratchFloats) {
+    if (chunk >= n_kv_cap) return SDPA_ERR_WORKSPACE;  // one split per (batch, head) is already too big
+    chunk *= 2;
+  }
+  if (int e = check_device()) return e;
+  int status = SDPA_OK;
+  float* scratch = static_scratch_for_current_device(&status);
+  if (!scratch) return status;
+  sdpa::DecodeParams p;
+  p.Q = (const __nv_bfloat16*)Q;
+  p.K = (const __nv_bfloat16*)K;
+  p.V = (const __nv_bfloat16*)V;
+  p.kv_lens = kv_lens;
+  p.H = heads;
+  p.n_cap = n_kv_cap;
+  p.chunk = (int)chunk;
+  p.n_split = (int)((n_kv_cap + chunk - 1) / chunk);
+  p.part_o = scratch;
+  p.part_lse = scratch + (size_t)bh * p.n_split * d_v;
+  p.O = (__nv_bfloat16*)O;
+  p.LSE = LSE;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = (cudaStream_t)stream;
+  dim3 grid((unsigned)p.n_split, (unsigned)heads, (unsigned)batch);
+  if (d_k == 64) {
+    sdpa::sdpa_decode_split_kernel<64><<<grid, sdpa::DECODE_THREADS, 0, s>>>(p);
+    sdpa::sdpa_decode_combine_kernel<64><<<(unsigned)bh, 64, 0, s>>>(p);
+  } else {
+    sdpa::sdpa_decode_split_kernel<128><<<grid, sdpa::DECODE_THREADS, 0, s>>>(p);
+    sdpa::sdpa_decode_combine_kernel<128><<<(unsigned)bh, 128, 0, s>>>(p);
+  }
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SDPA_OK : cuda_fail("decode launch (static scratch)", e);
+}
+
 extern "C" int sdpa_get_last_device_error(void* stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SDPA_ERR_CUDA;
   int v = 0;

@@ -28,7 +28,7 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
-        "sdpa_decode", "sdpa_decode_workspace_size", "sdpa_fwd", "sdpa_fwd_f32",
+        "sdpa_decode", "sdpa_decode_noalloc", "sdpa_decode_workspace_size", "sdpa_fwd", "sdpa_fwd_f32",
         "sdpa_get_last_device_error", "sdpa_status_string"])
 
 
