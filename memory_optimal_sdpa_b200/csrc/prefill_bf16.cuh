@@ -13,50 +13,66 @@
 //   warps 0-3  softmax warpgroup for query tile a (thread t owns TMEM lane = row t)
 //   warps 4-7  softmax warpgroup for query tile b
 //   warp  8    TMA producer: Q once, then K_j, V_j into a ring of shared-memory slots
-//   warp  9    MMA issuer (one thread) and TMEM owner
-//   warps 10-11 idle
+//   warp  9    MMA issuer for query tile a (one thread) and TMEM owner
+//   warp  10   MMA issuer for query tile b (one thread)
+//   warp  11   idle
 // Registers: each SM sub-partition holds 16K 32-bit registers and receives
 // one warp of every warpgroup, so the CTA launches at 168 per thread and then
-// moves registers from the producer/MMA warpgroup (down to 56) to the two
-// softmax warpgroups (up to 224): 2*224 + 56 <= 512 per sub-partition lane
-// slot, and 56*128 + 224*256 = 384*168 in total.
-// TMEM (512 columns): S_a [0,128), S_b [128,256), O_a [256,256+D), O_b [384,384+D).
-// P_x (bf16, two per column) overwrites the first 64 columns of S_x once the
-// softmax has read S_x; the next S_x MMA is issued after the P_x V MMA, and
-// tcgen05 MMAs from one thread run in issue order.
+// moves registers from the producer/MMA warpgroup (down to 72) to the two
+// softmax warpgroups (up to 216): 2*216 + 72 <= 512 per sub-partition lane
+// slot, and 72*128 + 216*256 = 384*168 in total.
 //
-// Per key tile j the issuer runs PV_a(j), S_a(j+1), PV_b(j), S_b(j+1), so that
-// one softmax warpgroup works while the tensor core serves the other.  The
-// online softmax keeps, per row, the running maximum m (in log2 units of the
-// scaled logits) and sum l; O and l are rescaled only when m grows by more
+// TMEM (512 columns).  d = 64: S_a [0,128), S_b [128,256), P_a [256,320),
+// P_b [320,384), O_a [384,448), O_b [448,512).  With P in its own columns the
+// softmax releases S_x as soon as it has loaded it, so the tensor core computes
+// S_x(j+1) while the softmax of tile j still runs.  d = 128: S_a, S_b, O_a
+// [256,384), O_b [384,512) fill the memory, so P_x (bf16, two per column)
+// overwrites the first 64 columns of S_x and the next S_x MMA is issued after
+// the P_x V MMA (tcgen05 MMAs from one thread run in issue order, and each
+// query tile's MMAs come from one thread).
+//
+// The online softmax keeps, per row, the running maximum m (in log2 units of
+// the scaled logits) and sum l; O and l are rescaled only when m grows by more
 // than 8 (a factor 256): O and l always share the same reference maximum, so
-// O/l is exact whatever reference is used, and fp32 cannot overflow.
+// O/l is exact whatever reference is used, and fp32 cannot overflow.  On tiles
+// without masked entries one column pair in SDPA_EXP2_POLY_EVERY takes its
+// exponentials on the FMA pipe (sm100::exp2_poly2) instead of the MUFU unit,
+// which is the softmax's bottleneck.
 #pragma once
 
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
 
+#ifndef SDPA_EXP2_POLY_EVERY
+#define SDPA_EXP2_POLY_EVERY 0
+#endif
+
 namespace sdpa {
 
 template <int D>
 struct PrefillCfg {
-  static constexpr int BM = 128;                        // query rows per tile
-  static constexpr int BN = 128;                        // key rows per tile
   static constexpr int TILE_BYTES = 128 * D * 2;        // one 128 x D bf16 tile
   static constexpr int BLOCK_BYTES = 128 * 64 * 2;      // one 128-row x 64-column swizzle block (16 KB)
   static constexpr int NSLOT = (D == 128) ? 4 : 8;      // K/V ring slots
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
-  static constexpr int NBAR = 1 + 2 * NSLOT + 2 + 2 + 2 + 1;
+  // q_full, full[NSLOT], empty[NSLOT], s_full[2], s_free[2], p_full[2], pv_done[2], o_full[2], turn[2], drain[2]
+  static constexpr int NBAR = 1 + 2 * NSLOT + 2 * 7;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;  // + tmem slot, abort flag, align slack
   static constexpr int THREADS = 384;
-  static constexpr int SOFTMAX_REGS = 224;
-  static constexpr int CONTROL_REGS = 56;
+  static constexpr int SOFTMAX_REGS = 216;
+  static constexpr int CONTROL_REGS = 72;
   static constexpr int LOAD_WARP = 8;
   static constexpr int MMA_WARP = 9;
   static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr bool P_SEPARATE = (D == 64);
+  __host__ __device__ static constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
+  __host__ __device__ static constexpr uint32_t col_p(int x) { return P_SEPARATE ? 256u + (uint32_t)x * 64u : col_s(x); }
+  __host__ __device__ static constexpr uint32_t col_o(int x) {
+    return P_SEPARATE ? 384u + (uint32_t)x * 64u : 256u + (uint32_t)x * 128u;
+  }
 };
 
 __device__ int g_sdpa_error;  // first device-side error since the last read (0 = none)
@@ -82,6 +98,53 @@ struct PrefillParams {
   float scale_log2;  // scale * log2(e), > 0
 };
 
+#ifndef SDPA_SM_INTPACK
+#define SDPA_SM_INTPACK 0
+#endif
+#ifndef SDPA_SM_TURN
+#define SDPA_SM_TURN 1
+#endif
+
+// Two finite, non-negative floats -> bf16x2 (lo in bits 0..15), rounded to nearest.
+// The conversion instruction shares the MUFU issue port with ex2, so the rounding is done
+// with integer adds and a byte permute instead (ties round away from zero, otherwise equal
+// to round-to-nearest-even).
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+#if SDPA_SM_INTPACK
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+#else
+  return sm100::pack_bf16x2(lo, hi);
+#endif
+}
+
+// Exponentials of one 128-score row: p = 2^(s*c2 - m), bf16 pairs into pk, returns sum p.
+// POLY: every SDPA_EXP2_POLY_EVERY-th pair on the FMA pipe (finite scores only).
+template <bool POLY>
+__device__ __forceinline__ float softmax_exp_row(const uint32_t (&s)[128], float c2, float m_use, uint32_t (&pk)[64]) {
+  using namespace sm100;
+  const float2 cc = make_float2(c2, c2), nm = make_float2(-m_use, -m_use);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const float2 xv = ffma2(make_float2(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), cc, nm);
+    float2 e;
+    if (POLY && SDPA_EXP2_POLY_EVERY > 0 && (i % (SDPA_EXP2_POLY_EVERY > 0 ? SDPA_EXP2_POLY_EVERY : 1)) ==
+                                                 SDPA_EXP2_POLY_EVERY - 1) {
+      e = exp2_poly2(xv);
+    } else {
+      e.x = ex2_approx(xv.x);
+      e.y = ex2_approx(xv.y);
+    }
+    if (i & 1)
+      acc1 = fadd2(acc1, e);
+    else
+      acc0 = fadd2(acc0, e);
+    pk[i] = pack_p(e.x, e.y);
+  }
+  const float2 a = fadd2(acc0, acc1);
+  return a.x + a.y;
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     sdpa_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -97,9 +160,12 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* full = bars + 1;
   uint64_t* empty = full + C::NSLOT;
   uint64_t* s_full = empty + C::NSLOT;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_full = p_full + 2;
-  uint64_t* drain = o_full + 2;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* o_full = pv_done + 2;
+  uint64_t* turn = o_full + 2;
+  uint64_t* drain = turn + 2;
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -118,14 +184,18 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < C::NSLOT; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 2);  // released by both MMA issuers
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
+      mbar_init(&s_free[x], 128);
       mbar_init(&p_full[x], 128);
+      mbar_init(&turn[x], 128);
+      mbar_init(&pv_done[x], 1);
       mbar_init(&o_full[x], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -139,6 +209,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
   bool timed_out = false;
   static_assert(C::SOFTMAX_REGS * 256 + C::CONTROL_REGS * 128 <= 168 * 384, "register split exceeds the launch");
+
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONTROL_REGS));
     if (warp == C::LOAD_WARP) {
@@ -148,9 +219,9 @@ __global__ void __launch_bounds__(384, 1)
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
-  #pragma unroll
+#pragma unroll
         for (int x = 0; x < 2; ++x)
-  #pragma unroll
+#pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
             tma_load_3d(sQ + x * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmQ, q_full, cb * 64, x ? r0b : r0a, bh);
         int issued = 0;
@@ -161,7 +232,7 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive_expect_tx(&full[slot], C::TILE_BYTES);
           const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
           uint8_t* dst = sKV + slot * C::TILE_BYTES;
-  #pragma unroll
+#pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
             tma_load_3d(dst + cb * C::BLOCK_BYTES, map, &full[slot], cb * 64, (idx >> 1) * 128, bh);
           issued = idx + 1;
@@ -172,74 +243,83 @@ __global__ void __launch_bounds__(384, 1)
             mbar_wait_drain(&full[idx % C::NSLOT], (uint32_t)(idx / C::NSLOT) & 1u);
         }
       }
-    } else if (warp == C::MMA_WARP) {
-      // ------------------------------------------------------------ MMA issuer
+    } else if (warp == C::MMA_WARP || warp == C::MMA_WARP + 1) {
+      // ------------------------------------------------------------ MMA issuers
+      // Query tile x's MMAs are issued by lane 0 of warp MMA_WARP + x, so the two
+      // instruction streams (and their barrier waits) proceed in parallel.  Within one
+      // stream tcgen05 MMAs execute in issue order, which is what lets P_x alias S_x.
+      const int x = warp - C::MMA_WARP;
+      const int tx = x ? tb : ta;
       if (lane == 0 && T > 0) {
-        const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-        const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
         constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // P (TMEM) x V (MN-major)
         const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
-
-        auto issue_S = [&](int x, int j) {  // S_x = Q_x K_j^T
-          const uint32_t qa = sQa + x * C::TILE_BYTES;
-          const uint32_t ka = sKVa + ((2 * j) % C::NSLOT) * C::TILE_BYTES;
-  #pragma unroll
+        // Descriptors are built once; every operand tile is then reached by adding its byte
+        // offset >> 4 to the start-address field (the low 14 bits; shared memory < 256 KB, so
+        // the add never carries out of the field).
+        const uint64_t dQ = smem_desc_sw128(sQa + x * C::TILE_BYTES, 16, 1024);  // K-major
+        const uint64_t dK = smem_desc_sw128(sKVa, 16, 1024);                     // K-major
+        const uint64_t dV = smem_desc_sw128(sKVa, C::BLOCK_BYTES, 1024);         // MN-major
+        const uint32_t tS = tmem + C::col_s(x), tP = tmem + C::col_p(x), tO = tmem + C::col_o(x);
+        auto issue_S = [&](int j) {  // S_x = Q_x K_j^T
+          const uint64_t b0 = dK + (uint64_t)((((2 * j) % C::NSLOT) * C::TILE_BYTES) >> 4);
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::BLOCK_BYTES + (kk & 3) * 32;
-            mma_ss(tS[x], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), idS,
-                   kk > 0 ? 1u : 0u);
+            const uint64_t off = (uint64_t)((((kk >> 2) * C::BLOCK_BYTES) + (kk & 3) * 32) >> 4);
+            mma_ss(tS, dQ + off, b0 + off, idS, kk > 0 ? 1u : 0u);
           }
         };
-        auto issue_PV = [&](int x, int j) {  // O_x += P_x V_j
-          const uint32_t va = sKVa + ((2 * j + 1) % C::NSLOT) * C::TILE_BYTES;
-  #pragma unroll
+        auto issue_PV = [&](int j) {  // O_x += P_x V_j
+          const uint64_t b0 = dV + (uint64_t)((((2 * j + 1) % C::NSLOT) * C::TILE_BYTES) >> 4);
+#pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk)
-            mma_ts(tO[x], tS[x] + kk * 8, smem_desc_sw128(va + kk * 2048, C::BLOCK_BYTES, 1024), idO,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tO, tP + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
         };
-        auto wait_slot = [&](int idx) {
-          return mbar_wait_bounded(&full[idx % C::NSLOT], (uint32_t)(idx / C::NSLOT) & 1u, abort_flag,
-                                   &timed_out);
+        auto wait_bar = [&](uint64_t* bar, int phase) {
+          const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
+          if (r) tc_fence_after_sync();
+          return r;
         };
+        auto wait_slot = [&](int idx) { return wait_bar(&full[idx % C::NSLOT], idx / C::NSLOT); };
 
-        bool ok = mbar_wait_bounded(q_full, 0, abort_flag, &timed_out) && wait_slot(0);
-        if (ok) {
-          tc_fence_after_sync();
-          if (ta > 0) { issue_S(0, 0); tc_commit(&s_full[0]); }
-          if (tb > 0) { issue_S(1, 0); tc_commit(&s_full[1]); }
-          tc_commit(&empty[0]);
+        bool ok = wait_bar(q_full, 0);
+        if (ok && tx > 0) {
+          if ((ok = wait_slot(0))) {
+            issue_S(0);
+            tc_commit(&s_full[x]);
+            tc_commit(&empty[0]);
+          }
         }
-        for (int j = 0; ok && j < T; ++j) {
-          if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
-          tc_fence_after_sync();
-          if (j < ta) {
-            if (!(ok = mbar_wait_bounded(&p_full[0], (uint32_t)j & 1u, abort_flag, &timed_out))) break;
-            tc_fence_after_sync();
-            issue_PV(0, j);
-            if (j == ta - 1) tc_commit(&o_full[0]);
+        for (int j = 0; ok && j < tx; ++j) {
+          if (C::P_SEPARATE && j + 1 < tx) {
+            // next S as soon as the softmax has read the current one
+            if (!(ok = wait_slot(2 * (j + 1)) && wait_bar(&s_free[x], j))) break;
+            issue_S(j + 1);
+            tc_commit(&s_full[x]);
+            tc_commit(&empty[(2 * (j + 1)) % C::NSLOT]);
           }
-          if (j + 1 < T) {
-            if (!(ok = wait_slot(2 * (j + 1)))) break;  // K_{j+1}
-            tc_fence_after_sync();
-            if (j + 1 < ta) { issue_S(0, j + 1); tc_commit(&s_full[0]); }
+          if (!(ok = wait_slot(2 * j + 1) && wait_bar(&p_full[x], j))) break;  // V_j and P_x(j)
+          issue_PV(j);
+          if (C::P_SEPARATE) tc_commit(&pv_done[x]);
+          if (j == tx - 1) tc_commit(&o_full[x]);
+          tc_commit(&empty[(2 * j + 1) % C::NSLOT]);
+          if (!C::P_SEPARATE && j + 1 < tx) {
+            // P_x aliases S_x: the next S_x is issued after P_x V (same stream, in order)
+            if (!(ok = wait_slot(2 * (j + 1)))) break;
+            issue_S(j + 1);
+            tc_commit(&s_full[x]);
+            tc_commit(&empty[(2 * (j + 1)) % C::NSLOT]);
           }
-          if (j < tb) {
-            if (!(ok = mbar_wait_bounded(&p_full[1], (uint32_t)j & 1u, abort_flag, &timed_out))) break;
-            tc_fence_after_sync();
-            issue_PV(1, j);
-            if (j == tb - 1) tc_commit(&o_full[1]);
-          }
-          tc_commit(&empty[(2 * j + 1) % C::NSLOT]);  // V_j slot free once both PV MMAs are done
-          if (j + 1 < T) {
-            if (j + 1 < tb) { issue_S(1, j + 1); tc_commit(&s_full[1]); }
-            tc_commit(&empty[(2 * (j + 1)) % C::NSLOT]);  // K_{j+1} slot
-          }
+        }
+        // Key tiles only the other query tile uses: release them once they have landed.
+        for (int idx = 2 * tx; ok && idx < 2 * T; ++idx) {
+          if (!(ok = wait_slot(idx))) break;
+          mbar_arrive(&empty[idx % C::NSLOT]);
         }
         // Every MMA and every commit issued above has landed before TMEM is released
         // and before the CTA's shared memory (which the commits arrive on) goes away.
-        tc_commit(drain);
-        mbar_wait_drain(drain, 0);
+        tc_commit(&drain[x]);
+        mbar_wait_drain(&drain[x], 0);
       }
     }
   } else {
@@ -250,8 +330,9 @@ __global__ void __launch_bounds__(384, 1)
     const int row = (x ? r0b : r0a) + t;
     const int tiles = x ? tb : ta;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tS = tmem + (x ? 128u : 0u) + lane_base;
-    const uint32_t tO = tmem + (x ? 384u : 256u) + lane_base;
+    const uint32_t tS = tmem + C::col_s(x) + lane_base;
+    const uint32_t tP = tmem + C::col_p(x) + lane_base;
+    const uint32_t tO = tmem + C::col_o(x) + lane_base;
     // last key this row may see
     int lim = p.n_kv - 1;
     if (CAUSAL) {
@@ -263,33 +344,60 @@ __global__ void __launch_bounds__(384, 1)
     float m_u = NEG_INF;  // running max of scale*log2(e)*s
     float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < tiles; ++j) {
-      if (!(ok = mbar_wait_bounded(&s_full[x], (uint32_t)j & 1u, abort_flag, &timed_out))) break;
-      tc_fence_after_sync();
+    // Waits ahead of warp-collective TMEM instructions: the whole warp proceeds or none of it.
+    auto wait_warp = [&](uint64_t* bar, int phase) {
+      const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
+      return __all_sync(0xffffffffu, r);
+    };
+    // The two softmax warpgroups take turns on the exponentials (the MUFU-bound part), so
+    // that one's TMEM traffic, row maxima and hand-offs -- and, with P aliasing S, its
+    // P V and next S MMAs -- overlap the other's exponentials.  Round j is tile a's turn,
+    // then tile b's; both run T = max(ta, tb) rounds (a round without a tile only passes
+    // the turn).  turn[x] completes phase j when the other warpgroup hands over; tile b
+    // hands tile a its first turn up front.
+    if (SDPA_SM_TURN && x == 1) mbar_arrive(&turn[0]);
+    for (int j = 0; ok && j < T; ++j) {
+      if (j >= tiles) {  // no key tile left for this query tile: only pass the turn
+        if (SDPA_SM_TURN) {
+          if (!(ok = wait_warp(&turn[x], j))) break;
+          mbar_arrive(&turn[x ^ 1]);
+        }
+        continue;
+      }
       uint32_t s[128];
-      {
-        uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
-        uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-        uint32_t(&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
-        uint32_t(&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
-        tmem_ld_32x32b_x32(tS + 0, s0);
-        tmem_ld_32x32b_x32(tS + 32, s1);
-        tmem_ld_32x32b_x32(tS + 64, s2);
-        tmem_ld_32x32b_x32(tS + 96, s3);
-        tmem_wait_ld();
-        reg_fence(s);
+      if (!(ok = wait_warp(&s_full[x], j))) break;
+      tc_fence_after_sync();
+      tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_wait_ld();
+      reg_fence(s);
+      if (C::P_SEPARATE) {  // S_x is in registers: the tensor core may overwrite it with S_x(j+1)
+        tc_fence_before_sync();
+        mbar_arrive(&s_free[x]);
       }
       const int kv0 = j * 128;
-      if (kv0 + 127 > lim) {
+      const bool masked = kv0 + 127 > lim;
+      if (masked) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (kv0 + c > lim) s[c] = __float_as_uint(NEG_INF);
       }
-      float mx = NEG_INF;
+      float mx;
+      {  // eight independent chains of 3-input maxima
+        float m[8];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        for (int k = 0; k < 8; ++k) m[k] = __uint_as_float(s[k]);
+#pragma unroll
+        for (int c = 8; c < 128; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m[k] = max3f(m[k], __uint_as_float(s[c + 2 * k]), __uint_as_float(s[c + 2 * k + 1]));
+        mx = max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+      }
       const float m_new = fmaxf(m_u, mx * c2);
       const bool need = m_new > m_u + 8.0f;
+      bool pv_waited = false;  // P_x V of the previous tile known complete (P_x and O_x free)
       if (__any_sync(0xffffffffu, need)) {
         float alpha = 1.f;
         if (m_new > m_u) {
@@ -297,7 +405,12 @@ __global__ void __launch_bounds__(384, 1)
           m_u = m_new;
           l *= alpha;
         }
-        if (j > 0) {  // O_x holds PV of earlier tiles (complete: S_x(j) was issued after them)
+        if (j > 0) {  // O_x holds P V of earlier tiles
+          if (C::P_SEPARATE) {
+            if (!(ok = wait_warp(&pv_done[x], j - 1))) break;
+            tc_fence_after_sync();
+            pv_waited = true;
+          }  // (aliased P: S_x(j) was issued after P_x V of tile j-1, so that is complete)
 #pragma unroll 1
           for (int cb = 0; cb < D; cb += 32) {
             uint32_t o[32];
@@ -310,25 +423,23 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
+      if (SDPA_SM_TURN && !(ok = wait_warp(&turn[x], j))) break;  // this warpgroup's turn on the exponentials
       const float m_use = (m_u == NEG_INF) ? 0.f : m_u;
-      float rs = 0.f;
       uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), c2, -m_use));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), c2, -m_use));
-        rs += p0 + p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
+      l += masked ? softmax_exp_row<false>(s, c2, m_use, pk) : softmax_exp_row<true>(s, c2, m_use, pk);
+      if (SDPA_SM_TURN) mbar_arrive(&turn[x ^ 1]);  // hand the exponentials over
+      if (C::P_SEPARATE && j > 0 && !pv_waited) {  // P_x V of tile j-1 still reads P_x
+        if (!(ok = wait_warp(&pv_done[x], j - 1))) break;
+        tc_fence_after_sync();
       }
-      l += rs;
-      tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_st_32x32b_x32(tP + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st_32x32b_x32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       tc_fence_before_sync();
       mbar_arrive(&p_full[x]);
     }
     // ---------------------------------------------------------------- epilogue
-    if (ok && tiles > 0) ok = mbar_wait_bounded(&o_full[x], 0, abort_flag, &timed_out);
+    if (ok && tiles > 0) ok = wait_warp(&o_full[x], 0);
     if (ok) {
       tc_fence_after_sync();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
