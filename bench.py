@@ -78,20 +78,26 @@ def profiled_traffic(summary, paths):
 
 
 class ClockSampler:
-    """nvidia-smi SM clocks and throttle reasons, sampled every 200 ms while running."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    """nvidia-smi SM clocks, utilisation and throttle reasons, sampled every 100 ms while running.
+
+    summary(t0, t1) reports the samples taken inside [t0, t1] (host wall clock; the timed
+    region) when there are any, else the samples of the whole window during which the GPU
+    was busy (utilisation > 0), and says which.
+    """
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,utilization.gpu,clocks_event_reasons.hw_slowdown,"
              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
              "clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.samples = []  # (unix time, sm_mhz, max_mhz, util, reasons)
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -100,11 +106,22 @@ class ClockSampler:
         return self
 
     def _read(self):
+        import datetime
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, mx, util = float(parts[2]), float(parts[3]), float(parts[4])
+            except ValueError:
+                continue
+            reasons = {n for n, f in zip(self.NAMES, parts[5:9]) if f.lower() in ("active", "1")}
+            self.samples.append((ts, sm, mx, util, reasons))
 
     def __exit__(self, *exc):
         if self.proc:
+            time.sleep(0.25)  # let the last sample land
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -112,24 +129,16 @@ class ClockSampler:
                 self.proc.kill()
             self.thread.join(timeout=2)
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for name, flag in zip(names, parts[4:8]):
-                if flag.lower() in ("active", "1"):
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+    def summary(self, t0=None, t1=None):
+        inside = [x for x in self.samples if t0 is not None and t0 - 0.05 <= x[0] <= t1 + 0.05]
+        chosen, where = inside, "timed region"
+        if not chosen:
+            chosen, where = [x for x in self.samples if x[3] > 0], "busy samples of the bench window"
+        if not chosen:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "from": "none"}
+        reasons = sorted(set().union(*(x[4] for x in chosen)))
+        return {"sm_mhz": float(np.median([x[1] for x in chosen])), "sm_max_mhz": chosen[-1][2],
+                "reasons": reasons, "samples": len(chosen), "from": where}
 
 
 # ---------------------------------------------------------------------------------------------- distributed
@@ -224,6 +233,8 @@ def run_ours(args):
         for w, (o, lse) in zip(works, outs):
             sdpa.fwd(qq, kk, vv, causal=w.causal, scale=w.scale_f32, o=o, lse=lse, stream=stream)
 
+    clocks = ClockSampler(local_rank).__enter__()  # sampled from warm-up through the end-to-end loop
+    time.sleep(0.3)
     for _ in range(args.warmup):
         step()
     if sdpa.get_last_device_error() != sdpa.SDPA_OK:
@@ -234,14 +245,15 @@ def run_ours(args):
           for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clocks:
-        for s in range(args.steps):
-            flush.zero_()
-            for (a, b), w, (o, lse) in zip(ev[s], works, outs):
-                a.record(stream)
-                sdpa.fwd(q, k, v, causal=w.causal, scale=w.scale_f32, o=o, lse=lse, stream=stream)
-                b.record(stream)
-        torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for s in range(args.steps):
+        flush.zero_()
+        for (a, b), w, (o, lse) in zip(ev[s], works, outs):
+            a.record(stream)
+            sdpa.fwd(q, k, v, causal=w.causal, scale=w.scale_f32, o=o, lse=lse, stream=stream)
+            b.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
     barrier()
     per_launch = np.array([[a.elapsed_time(b) for (a, b) in row] for row in ev]) / 1e3  # seconds [step, launch]
     local_t = float(per_launch.sum())
@@ -293,6 +305,7 @@ def run_ours(args):
         b.record(stream)
         torch.cuda.synchronize()
         e_times.append(a.elapsed_time(b) / 1e3)
+    clocks.__exit__(None, None, None)
     e_max, e_units = aggregate(float(np.sum(e_times)), step_flops * args.steps)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
     d2h = sum(po.numel() * po.element_size() + pl.numel() * pl.element_size() for po, pl in ho)
@@ -316,7 +329,7 @@ def run_ours(args):
         "roofline": roof,
         "gpu_launches": args.steps * len(works),
         "e2e": e2e,
-        "clocks": clocks.summary(),
+        "clocks": clocks.summary(t_wall0, t_wall1),
     }
     if decode is not None:
         line["decode"] = decode

@@ -436,7 +436,11 @@ __global__ void __launch_bounds__(384, 1)
       tmem_st_32x32b_x32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(&p_full[x]);
+#ifdef SDPA_FAULT_DROP_ARRIVE
+      // Test builds only: tile b never reports its first P, so its MMA issuer's wait runs out.
+      if (!(x == 1 && j == 0))
+#endif
+        mbar_arrive(&p_full[x]);
     }
     // ---------------------------------------------------------------- epilogue
     if (ok && tiles > 0) ok = wait_warp(&o_full[x], 0);
