@@ -40,6 +40,9 @@ def lib():
                                        _f64p, _f64p]
         L.oracle_sdpa_rows.argtypes = [_f32p, _f32p, _f32p, I64, I64, I64, I32, I32, D, I32, _i64p, I64,
                                        _f64p, _f64p, I32]
+        L.oracle_sdpa_rows_window.argtypes = [_f32p, _f32p, _f32p, I64, I64, I64, I32, I32, D, I64, I64, _i64p,
+                                               I64, _f64p, _f64p, I32]
+        L.oracle_sdpa_rows_window.restype = ctypes.c_int
         L.oracle_decode.argtypes = [_f32p, _f32p, _f32p, _i32p, I64, I64, I64, I32, I32, D, _i64p, I64,
                                     _f64p, _f64p, I32]
         for f in (L.oracle_scores, L.oracle_softmax_rows, L.oracle_softmax_naive, L.oracle_sdpa_full,
@@ -123,6 +126,28 @@ def sdpa_rows(q, k, v, scale, causal=False, rows=None, threads=None):
     _check(lib().oracle_sdpa_rows(qp, kp, vp, bh, n_q, n_kv, d_k, d_v, scale, int(causal), rp, n_rows,
                                   O.ctypes.data_as(_f64p), L.ctypes.data_as(_f64p),
                                   threads or threads_available()), "oracle_sdpa_rows")
+    return O, L
+
+
+def sdpa_rows_window(q, k, v, scale, left, right, rows=None, threads=None):
+    """Like sdpa_rows with a local window: row i (key position p = i + n_kv - n_q) sees keys
+    p - left <= j <= p + right; a negative bound leaves that side open."""
+    lead = q.shape[:-2]
+    n_q, d_k = q.shape[-2:]
+    n_kv, d_v = v.shape[-2:]
+    bh = int(np.prod(lead, dtype=np.int64)) if lead else 1
+    q, qp = _f32(q)
+    k, kp = _f32(k)
+    v, vp = _f32(v)
+    if rows is None:
+        rp, n_rows = None, n_q
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        rp, n_rows = rows.ctypes.data_as(_i64p), rows.shape[0]
+    O = np.empty(lead + (n_rows, d_v)); L = np.empty(lead + (n_rows,))
+    _check(lib().oracle_sdpa_rows_window(qp, kp, vp, bh, n_q, n_kv, d_k, d_v, scale, int(left), int(right), rp,
+                                         n_rows, O.ctypes.data_as(_f64p), L.ctypes.data_as(_f64p),
+                                         threads or threads_available()), "oracle_sdpa_rows_window")
     return O, L
 
 

@@ -20,12 +20,23 @@ bool allowed(int64_t i, int64_t j, int64_t n_q, int64_t n_kv, int causal) {
   return j <= i + (n_kv - n_q);  // bottom-right aligned causal mask
 }
 
+// Local window: query row i sits at key position p = i + (n_kv - n_q) and sees keys
+// p - left <= j <= p + right; a negative bound means that side is unbounded.
+bool allowed_window(int64_t i, int64_t j, int64_t n_q, int64_t n_kv, int64_t left, int64_t right) {
+  const int64_t pos = i + (n_kv - n_q);
+  if (left >= 0 && j < pos - left) return false;
+  if (right >= 0 && j > pos + right) return false;
+  return true;
+}
+
 // s_j = scale * q . k_j for every key j of one slice; -inf where masked.
+// causal < 0 selects the local window (left, right) instead of the causal flag.
 void score_row(const float* Q, const float* K, int64_t i, int64_t n_q, int64_t n_kv, int d_k,
-               double scale, int causal, double* s) {
+               double scale, int causal, double* s, int64_t left = -1, int64_t right = -1) {
   const float* q = Q + i * d_k;
   for (int64_t j = 0; j < n_kv; ++j) {
-    if (!allowed(i, j, n_q, n_kv, causal)) {
+    const bool ok = causal >= 0 ? allowed(i, j, n_q, n_kv, causal) : allowed_window(i, j, n_q, n_kv, left, right);
+    if (!ok) {
       s[j] = kNegInf;
       continue;
     }
@@ -192,6 +203,25 @@ extern "C" int oracle_decode(const float* Q, const float* K, const float* V, con
     // one query row (row 0 of a 1-row slice) against the first n keys of the cache
     score_row(Q + bh * d_k, K + bh * n_cap * d_k, 0, 1, n, d_k, scale, 0, s.data());
     attend_row(s.data(), V + bh * n_cap * d_v, n, d_v, O + p * d_v, LSE + p);
+  });
+  return 0;
+}
+
+extern "C" int oracle_sdpa_rows_window(const float* Q, const float* K, const float* V, int64_t bh, int64_t n_q,
+                                       int64_t n_kv, int d_k, int d_v, double scale, int64_t left, int64_t right,
+                                       const int64_t* rows, int64_t n_rows, double* O, double* LSE, int threads) {
+  if (bh < 0 || n_q < 0 || n_kv <= 0 || d_k <= 0 || d_v <= 0 || n_rows < 0) return -1;
+  if (!rows && n_rows != n_q) return -1;
+  if (bh == 0 || n_rows == 0) return 0;
+  if (!Q || !K || !V || !O || !LSE) return -1;
+  for (int64_t r = 0; rows && r < n_rows; ++r)
+    if (rows[r] < 0 || rows[r] >= n_q) return -1;
+  parallel_for(bh * n_rows, threads, [&](int64_t t) {
+    int64_t b = t / n_rows, r = t % n_rows;
+    int64_t i = rows ? rows[r] : r;
+    std::vector<double> s((size_t)n_kv);
+    score_row(Q + b * n_q * d_k, K + b * n_kv * d_k, i, n_q, n_kv, d_k, scale, -1, s.data(), left, right);
+    attend_row(s.data(), V + b * n_kv * d_v, n_kv, d_v, O + t * d_v, LSE + t);
   });
   return 0;
 }

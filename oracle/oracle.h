@@ -15,6 +15,7 @@
  * For one query row i of one (batch, head) slice:
  *   allowed(i, j) = true                          non-causal
  *                 = j <= i + (n_kv - n_q)         causal (bottom-right aligned)
+ *                 = p - left <= j <= p + right    local window, p = i + (n_kv - n_q)
  *   s_ij  = scale * sum_k Q[i,k] K[j,k]           (allowed j only)
  *   m_i   = max_j s_ij
  *   e_ij  = exp(s_ij - m_i),  l_i = sum_j e_ij
@@ -63,6 +64,13 @@ int oracle_sdpa_full(const float* Q, const float* K, const float* V, int64_t n_q
 int oracle_sdpa_rows(const float* Q, const float* K, const float* V, int64_t bh, int64_t n_q,
                      int64_t n_kv, int d_k, int d_v, double scale, int causal, const int64_t* rows,
                      int64_t n_rows, double* O, double* LSE, int threads);
+
+/* oracle_sdpa_rows with a local window instead of the causal flag: query row i sits at key
+   position p = i + (n_kv - n_q) and sees keys p - left <= j <= p + right; a negative bound
+   leaves that side open ((-1, 0) is causal, (-1, -1) is full attention). */
+int oracle_sdpa_rows_window(const float* Q, const float* K, const float* V, int64_t bh, int64_t n_q,
+                            int64_t n_kv, int d_k, int d_v, double scale, int64_t left, int64_t right,
+                            const int64_t* rows, int64_t n_rows, double* O, double* LSE, int threads);
 
 /* Decode: one query row per (b, h) against the first lens[b] keys of a cache.
    Q [B, H, d_k]; K [B, H, n_cap, d_k]; V [B, H, n_cap, d_v]; O [B, H, d_v]; LSE [B, H].

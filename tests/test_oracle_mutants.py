@@ -22,6 +22,9 @@ MUTANTS = {
     "no_normalisation": ("for (int c = 0; c < d_v; ++c) o[c] /= l;", ""),
     "v_row_index_wrong": ("const float* v = V + j * d_v;", "const float* v = V + (n_kv - 1 - j) * d_v;"),
     "q_k_swapped_rows": ("const float* k = K + j * d_k;", "const float* k = K + (j % (i + 1)) * d_k;"),
+    "window_left_off_by_one": ("if (left >= 0 && j < pos - left) return false;", "if (left >= 0 && j <= pos - left) return false;"),
+    "window_right_ignored": ("if (right >= 0 && j > pos + right) return false;", ""),
+    "window_position_top_left": ("const int64_t pos = i + (n_kv - n_q);", "const int64_t pos = i;"),
 }
 
 

@@ -265,3 +265,63 @@ def test_rejects_bad_arguments():
     with pytest.raises(ValueError):
         oracle.decode(np.zeros((1, 1, 4), np.float32), np.zeros((1, 1, 4, 4), np.float32),
                       np.zeros((1, 1, 4, 4), np.float32), np.array([5], np.int32), 1.0)
+
+
+# ------------------------------------------------------------------------------------------- local windows
+# Sliding (local) windows generalise the causal mask: row i, at key position p = i + (n_kv - n_q),
+# sees keys p - left <= j <= p + right (the windowed attention the 2-simplicial article uses to
+# bound cost, applied here to ordinary attention).
+def test_window_zero_width_returns_own_v_row():
+    n_q, n_kv, d = 5, 9, 6
+    q = RNG.integers(-3, 4, size=(n_q, d)).astype(np.float32)
+    k = RNG.integers(-3, 4, size=(n_kv, d)).astype(np.float32)
+    v = RNG.standard_normal((n_kv, 4)).astype(np.float32)
+    O, L = oracle.sdpa_rows_window(q, k, v, 0.5, 0, 0)
+    for i in range(n_q):
+        p = i + n_kv - n_q
+        np.testing.assert_array_equal(O[i], v[p].astype(np.float64))
+        assert L[i] == 0.5 * float(q[i].astype(np.int64) @ k[p].astype(np.int64))
+
+
+def test_window_reduces_to_full_and_causal():
+    n_q, n_kv, d = 7, 11, 5
+    q, k = RNG.standard_normal((n_q, d)).astype(np.float32), RNG.standard_normal((n_kv, d)).astype(np.float32)
+    v = RNG.standard_normal((n_kv, 3)).astype(np.float32)
+    for (left, right), causal in (((-1, -1), False), ((-1, 0), True), ((n_kv, n_kv), False), ((n_kv, 0), True)):
+        Ow, Lw = oracle.sdpa_rows_window(q, k, v, 0.4, left, right)
+        O, L = oracle.sdpa_rows(q, k, v, 0.4, causal)
+        np.testing.assert_array_equal(Ow, O)
+        np.testing.assert_array_equal(Lw, L)
+
+
+def _brute_force_window(q, k, v, scale, left, right):
+    n_q, n_kv = len(q), len(k)
+    O, L = [], []
+    for i in range(n_q):
+        p = i + n_kv - n_q
+        ws = []
+        for j in range(n_kv):
+            if (left >= 0 and j < p - left) or (right >= 0 and j > p + right):
+                ws.append(0.0)
+                continue
+            ws.append(math.exp(scale * math.fsum(float(a) * float(b) for a, b in zip(q[i], k[j]))))
+        z = math.fsum(ws)
+        if z == 0:
+            O.append([0.0] * len(v[0])); L.append(-math.inf); continue
+        O.append([math.fsum(w * float(v[j][c]) for j, w in enumerate(ws)) / z for c in range(len(v[0]))])
+        L.append(math.log(z))
+    return np.array(O), np.array(L)
+
+
+@pytest.mark.parametrize("left,right", [(0, 0), (2, 0), (3, 1), (-1, 2), (1, -1), (4, 4)])
+@pytest.mark.parametrize("n_q,n_kv", [(6, 6), (4, 9), (9, 4)])
+def test_window_brute_force(n_q, n_kv, left, right):
+    q = RNG.uniform(-1, 1, (n_q, 4)).astype(np.float32)
+    k = RNG.uniform(-1, 1, (n_kv, 4)).astype(np.float32)
+    v = RNG.standard_normal((n_kv, 3)).astype(np.float32)
+    O, L = oracle.sdpa_rows_window(q, k, v, 1.1, left, right)
+    Ob, Lb = _brute_force_window(q, k, v, 1.1, left, right)
+    np.testing.assert_allclose(O, Ob, rtol=1e-13, atol=1e-14)
+    assert (np.isneginf(L) == np.isneginf(Lb)).all()
+    fin = np.isfinite(Lb)
+    np.testing.assert_allclose(L[fin], Lb[fin], rtol=0, atol=1e-13)
