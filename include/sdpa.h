@@ -78,6 +78,24 @@ SDPA_API int sdpa_fwd(const void* Q, const void* K, const void* V, void* O, floa
              int n_q, int n_kv, int d_k, int d_v, float scale, int causal, void* stream);
 
 /*
+ * sdpa_fwd_window -- sdpa_fwd with a local (sliding) window instead of the causal flag.
+ *
+ * Query row i sits at key position p = i + (n_kv - n_q) (bottom-right alignment, as for
+ * causal masking) and sees keys j with p - window_left <= j <= p + window_right.  -1 leaves
+ * that side open: (-1, 0) is causal, (-1, -1) full attention, (w, 0) a causal window of
+ * w + 1 keys.  Key tiles wholly outside every row's window are skipped, so the work is
+ * proportional to the window, not to n_kv.  Rows whose window holds no key get O = 0 and
+ * LSE = -inf.  Windowed attention as the way to bound the cost of long sequences follows the
+ * 2-simplicial article (szyisi.cn, "model design": sliding windows w1, w2 over the sequence);
+ * here the window is the one-dimensional one of ordinary attention.
+ * Other arguments, layouts, alignment and errors as sdpa_fwd; window_left and window_right
+ * must be >= -1 (else SDPA_ERR_INVALID_ARG).
+ */
+SDPA_API int sdpa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* LSE, int batch,
+                             int heads, int n_q, int n_kv, int d_k, int d_v, float scale, int window_left,
+                             int window_right, void* stream);
+
+/*
  * sdpa_fwd_f32 -- fp32 prefill on the CUDA cores (FMA pipes); same semantics as
  * sdpa_fwd with float tensors.  1 <= d_k, d_v <= 128.  Scores, softmax
  * weights and the output sum are all fp32 (no tensor cores: TF32 would lose

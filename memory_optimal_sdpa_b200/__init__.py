@@ -25,6 +25,8 @@ lib = ctypes.CDLL(LIB_PATH)
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 lib.sdpa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
 lib.sdpa_fwd.restype = _i
+lib.sdpa_fwd_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp]
+lib.sdpa_fwd_window.restype = _i
 lib.sdpa_fwd_f32.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
 lib.sdpa_fwd_f32.restype = _i
 lib.sdpa_decode_workspace_size.argtypes = [_i, _i, _i, _i]
@@ -91,6 +93,18 @@ def fwd(q, k, v, causal=False, scale=None, o=None, lse=None, want_lse=True, stre
     o, lse = _outputs(q, n_q, d_v, q.dtype, o, lse, want_lse)
     _check(lib.sdpa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, n_q, n_kv, d_k, d_v,
                         float(scale), int(bool(causal)), _stream(stream)), "sdpa_fwd")
+    return o, lse
+
+
+def fwd_window(q, k, v, window_left, window_right, scale=None, o=None, lse=None, want_lse=True, stream=None):
+    """bf16 prefill with a local window: row i (key position p = i + n_kv - n_q) sees keys
+    p - window_left .. p + window_right; -1 leaves a side open."""
+    B, H, n_q, d_k = q.shape
+    n_kv, d_v = v.shape[2], v.shape[3]
+    scale = 1.0 / math.sqrt(d_k) if scale is None else scale
+    o, lse = _outputs(q, n_q, d_v, q.dtype, o, lse, want_lse)
+    _check(lib.sdpa_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, n_q, n_kv, d_k, d_v,
+                               float(scale), int(window_left), int(window_right), _stream(stream)), "sdpa_fwd_window")
     return o, lse
 
 

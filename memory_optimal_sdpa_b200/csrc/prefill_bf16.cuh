@@ -79,24 +79,31 @@ __device__ int g_sdpa_error;  // first device-side error since the last read (0 
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_sdpa_error, 0, code); }
 
-// Number of 128-row key tiles query tile [r0, r0+128) must visit.
-__host__ __device__ inline int prefill_kv_tiles(int r0, int n_q, int n_kv, bool causal) {
-  if (r0 >= n_q) return 0;
-  const int total = (n_kv + 127) / 128;
-  if (!causal) return total;
-  const int last_row = (r0 + 127 < n_q - 1) ? r0 + 127 : n_q - 1;
-  const long long max_key = (long long)last_row + n_kv - n_q;  // bottom-right aligned
-  if (max_key < 0) return 0;
-  const int t = (int)(max_key / 128) + 1;
-  return t < total ? t : total;
-}
-
 struct PrefillParams {
   __nv_bfloat16* O;
   float* LSE;
   int n_q, n_kv, bh_count, n_pairs;
   float scale_log2;  // scale * log2(e), > 0
+  // Local window (mask mode 2 only): query row i (key position p = i + n_kv - n_q)
+  // sees keys p - win_left <= j <= p + win_right; -1 leaves a side open.
+  int win_left, win_right;
 };
+
+// Key tiles [first, first + count) that query tile [r0, r0 + 128) must visit.
+__host__ __device__ inline void prefill_kv_range(int r0, int n_q, int n_kv, int win_left, int win_right,
+                                                 int* first, int* count) {
+  *first = 0;
+  *count = 0;
+  if (r0 >= n_q) return;
+  const int last_row = (r0 + 127 < n_q - 1) ? r0 + 127 : n_q - 1;
+  const long long off = (long long)n_kv - n_q;  // bottom-right alignment
+  long long hi = n_kv - 1, lo = 0;
+  if (win_right >= 0 && last_row + off + win_right < hi) hi = last_row + off + win_right;
+  if (win_left >= 0 && r0 + off - win_left > lo) lo = r0 + off - win_left;
+  if (hi < lo) return;
+  *first = (int)(lo / 128);
+  *count = (int)(hi / 128) - *first + 1;
+}
 
 #ifndef SDPA_SM_INTPACK
 #define SDPA_SM_INTPACK 0
@@ -145,7 +152,9 @@ __device__ __forceinline__ float softmax_exp_row(const uint32_t (&s)[128], float
   return a.x + a.y;
 }
 
-template <int D, bool CAUSAL>
+// MASK: 0 full attention, 1 causal (bottom-right aligned), 2 local window (p.win_left, p.win_right).
+// Modes 0 and 1 fix the bounds at compile time, so their key ranges and masks fold to constants.
+template <int D, int MASK>
 __global__ void __launch_bounds__(384, 1)
     sdpa_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -176,9 +185,16 @@ __global__ void __launch_bounds__(384, 1)
   const int bh = blockIdx.x % p.bh_count;
   const int pair = p.n_pairs - 1 - (int)(blockIdx.x / p.bh_count);
   const int r0a = pair * 256, r0b = pair * 256 + 128;
-  const int ta = prefill_kv_tiles(r0a, p.n_q, p.n_kv, CAUSAL);
-  const int tb = prefill_kv_tiles(r0b, p.n_q, p.n_kv, CAUSAL);
-  const int T = ta > tb ? ta : tb;
+  const int win_left = MASK == 2 ? p.win_left : -1;
+  const int win_right = MASK == 2 ? p.win_right : (MASK == 1 ? 0 : -1);
+  int fa, ta, fb, tb;  // first key tile and tile count of query tiles a and b
+  prefill_kv_range(r0a, p.n_q, p.n_kv, win_left, win_right, &fa, &ta);
+  prefill_kv_range(r0b, p.n_q, p.n_kv, win_left, win_right, &fb, &tb);
+  const int T = ta > tb ? ta : tb;  // softmax rounds
+  // Key tiles loaded: J0 .. J0 + TL - 1, the union of both ranges (ring index 2 (j - J0) for K_j, +1 for V_j).
+  const int J0 = ta == 0 ? fb : (tb == 0 ? fa : (fa < fb ? fa : fb));
+  const int J1 = ta == 0 ? fb + tb - 1 : (tb == 0 ? fa + ta - 1 : (fa + ta > fb + tb ? fa + ta - 1 : fb + tb - 1));
+  const int TL = (ta == 0 && tb == 0) ? 0 : J1 - J0 + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -214,7 +230,7 @@ __global__ void __launch_bounds__(384, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONTROL_REGS));
     if (warp == C::LOAD_WARP) {
       // ------------------------------------------------------------ TMA producer
-      if (lane == 0 && T > 0) {
+      if (lane == 0 && TL > 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
@@ -225,7 +241,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int cb = 0; cb < D / 64; ++cb)
             tma_load_3d(sQ + x * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmQ, q_full, cb * 64, x ? r0b : r0a, bh);
         int issued = 0;
-        for (int idx = 0; idx < 2 * T; ++idx) {
+        for (int idx = 0; idx < 2 * TL; ++idx) {
           const int slot = idx % C::NSLOT;
           const uint32_t ph = (uint32_t)(idx / C::NSLOT) & 1u;
           if (!mbar_wait_bounded(&empty[slot], ph ^ 1u, abort_flag, &timed_out)) break;
@@ -234,7 +250,7 @@ __global__ void __launch_bounds__(384, 1)
           uint8_t* dst = sKV + slot * C::TILE_BYTES;
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
-            tma_load_3d(dst + cb * C::BLOCK_BYTES, map, &full[slot], cb * 64, (idx >> 1) * 128, bh);
+            tma_load_3d(dst + cb * C::BLOCK_BYTES, map, &full[slot], cb * 64, (J0 + (idx >> 1)) * 128, bh);
           issued = idx + 1;
         }
         if (*abort_flag) {  // let the copies already in flight land before the CTA exits
@@ -250,7 +266,8 @@ __global__ void __launch_bounds__(384, 1)
       // stream tcgen05 MMAs execute in issue order, which is what lets P_x alias S_x.
       const int x = warp - C::MMA_WARP;
       const int tx = x ? tb : ta;
-      if (lane == 0 && T > 0) {
+      const int lead = tx ? (x ? fb : fa) - J0 : TL;  // loaded key tiles before this query tile's first
+      if (lane == 0 && TL > 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
         constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // P (TMEM) x V (MN-major)
         const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
@@ -261,19 +278,20 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t dK = smem_desc_sw128(sKVa, 16, 1024);                     // K-major
         const uint64_t dV = smem_desc_sw128(sKVa, C::BLOCK_BYTES, 1024);         // MN-major
         const uint32_t tS = tmem + C::col_s(x), tP = tmem + C::col_p(x), tO = tmem + C::col_o(x);
-        auto issue_S = [&](int j) {  // S_x = Q_x K_j^T
-          const uint64_t b0 = dK + (uint64_t)((((2 * j) % C::NSLOT) * C::TILE_BYTES) >> 4);
+        // r: this query tile's r-th key tile, the (lead + r)-th one loaded
+        auto issue_S = [&](int r) {  // S_x = Q_x K^T
+          const uint64_t b0 = dK + (uint64_t)((((2 * (lead + r)) % C::NSLOT) * C::TILE_BYTES) >> 4);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = (uint64_t)((((kk >> 2) * C::BLOCK_BYTES) + (kk & 3) * 32) >> 4);
             mma_ss(tS, dQ + off, b0 + off, idS, kk > 0 ? 1u : 0u);
           }
         };
-        auto issue_PV = [&](int j) {  // O_x += P_x V_j
-          const uint64_t b0 = dV + (uint64_t)((((2 * j + 1) % C::NSLOT) * C::TILE_BYTES) >> 4);
+        auto issue_PV = [&](int r) {  // O_x += P_x V
+          const uint64_t b0 = dV + (uint64_t)((((2 * (lead + r) + 1) % C::NSLOT) * C::TILE_BYTES) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk)
-            mma_ts(tO, tP + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tO, tP + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idO, (r > 0 || kk > 0) ? 1u : 0u);
         };
         auto wait_bar = [&](uint64_t* bar, int phase) {
           const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
@@ -283,36 +301,41 @@ __global__ void __launch_bounds__(384, 1)
         auto wait_slot = [&](int idx) { return wait_bar(&full[idx % C::NSLOT], idx / C::NSLOT); };
 
         bool ok = wait_bar(q_full, 0);
+        // Key tiles only the other query tile uses are released, in order, once they have landed.
+        for (int idx = 0; ok && idx < 2 * lead; ++idx) {
+          if (!(ok = wait_slot(idx))) break;
+          mbar_arrive(&empty[idx % C::NSLOT]);
+        }
+        const int k0 = 2 * lead;  // ring index of this query tile's first K
         if (ok && tx > 0) {
-          if ((ok = wait_slot(0))) {
+          if ((ok = wait_slot(k0))) {
             issue_S(0);
             tc_commit(&s_full[x]);
-            tc_commit(&empty[0]);
+            tc_commit(&empty[k0 % C::NSLOT]);
           }
         }
         for (int j = 0; ok && j < tx; ++j) {
           if (C::P_SEPARATE && j + 1 < tx) {
             // next S as soon as the softmax has read the current one
-            if (!(ok = wait_slot(2 * (j + 1)) && wait_bar(&s_free[x], j))) break;
+            if (!(ok = wait_slot(k0 + 2 * (j + 1)) && wait_bar(&s_free[x], j))) break;
             issue_S(j + 1);
             tc_commit(&s_full[x]);
-            tc_commit(&empty[(2 * (j + 1)) % C::NSLOT]);
+            tc_commit(&empty[(k0 + 2 * (j + 1)) % C::NSLOT]);
           }
-          if (!(ok = wait_slot(2 * j + 1) && wait_bar(&p_full[x], j))) break;  // V_j and P_x(j)
+          if (!(ok = wait_slot(k0 + 2 * j + 1) && wait_bar(&p_full[x], j))) break;  // V and P_x of tile j
           issue_PV(j);
           if (C::P_SEPARATE) tc_commit(&pv_done[x]);
           if (j == tx - 1) tc_commit(&o_full[x]);
-          tc_commit(&empty[(2 * j + 1) % C::NSLOT]);
+          tc_commit(&empty[(k0 + 2 * j + 1) % C::NSLOT]);
           if (!C::P_SEPARATE && j + 1 < tx) {
             // P_x aliases S_x: the next S_x is issued after P_x V (same stream, in order)
-            if (!(ok = wait_slot(2 * (j + 1)))) break;
+            if (!(ok = wait_slot(k0 + 2 * (j + 1)))) break;
             issue_S(j + 1);
             tc_commit(&s_full[x]);
-            tc_commit(&empty[(2 * (j + 1)) % C::NSLOT]);
+            tc_commit(&empty[(k0 + 2 * (j + 1)) % C::NSLOT]);
           }
         }
-        // Key tiles only the other query tile uses: release them once they have landed.
-        for (int idx = 2 * tx; ok && idx < 2 * T; ++idx) {
+        for (int idx = k0 + 2 * tx; ok && idx < 2 * TL; ++idx) {
           if (!(ok = wait_slot(idx))) break;
           mbar_arrive(&empty[idx % C::NSLOT]);
         }
@@ -333,11 +356,13 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS = tmem + C::col_s(x) + lane_base;
     const uint32_t tP = tmem + C::col_p(x) + lane_base;
     const uint32_t tO = tmem + C::col_o(x) + lane_base;
-    // last key this row may see
-    int lim = p.n_kv - 1;
-    if (CAUSAL) {
-      const long long c = (long long)row + p.n_kv - p.n_q;
-      if (c < lim) lim = (int)(c < -1 ? -1 : c);
+    // keys this row may see: lo .. lim
+    const int first = x ? fb : fa;
+    int lim = p.n_kv - 1, lo = 0;
+    {
+      const long long pos = (long long)row + p.n_kv - p.n_q;
+      if (win_right >= 0 && pos + win_right < lim) lim = (int)(pos + win_right < -1 ? -1 : pos + win_right);
+      if (win_left >= 0 && pos - win_left > 0) lo = (int)(pos - win_left > p.n_kv ? p.n_kv : pos - win_left);
     }
     const float c2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
@@ -377,12 +402,12 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_before_sync();
         mbar_arrive(&s_free[x]);
       }
-      const int kv0 = j * 128;
-      const bool masked = kv0 + 127 > lim;
+      const int kv0 = (first + j) * 128;
+      const bool masked = kv0 + 127 > lim || kv0 < lo;
       if (masked) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (kv0 + c > lim) s[c] = __float_as_uint(NEG_INF);
+          if (kv0 + c > lim || kv0 + c < lo) s[c] = __float_as_uint(NEG_INF);
       }
       float mx;
       {  // eight independent chains of 3-input maxima

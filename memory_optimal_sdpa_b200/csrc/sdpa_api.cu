@@ -82,11 +82,11 @@ int check_device() {
   return SDPA_OK;
 }
 
-template <int D, bool CAUSAL>
+template <int D, int MASK>
 int launch_prefill(const void* Q, const void* K, const void* V, void* O, float* LSE, int bh, int n_q,
-                   int n_kv, float scale, cudaStream_t stream) {
+                   int n_kv, float scale, int win_left, int win_right, cudaStream_t stream) {
   using Cfg = sdpa::PrefillCfg<D>;
-  auto kern = sdpa::sdpa_fwd_bf16_kernel<D, CAUSAL>;
+  auto kern = sdpa::sdpa_fwd_bf16_kernel<D, MASK>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -104,6 +104,8 @@ int launch_prefill(const void* Q, const void* K, const void* V, void* O, float* 
   p.bh_count = bh;
   p.n_pairs = (n_q + 255) / 256;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.win_left = win_left;
+  p.win_right = win_right;
   const long long grid = (long long)bh * p.n_pairs;
   kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   const cudaError_t e = cudaGetLastError();
@@ -113,7 +115,7 @@ int launch_prefill(const void* Q, const void* K, const void* V, void* O, float* 
       std::fprintf(stderr,
                    "sdpa: prefill<%d,%d> regs %d maxThreads %d static smem %zu max dyn smem %d local %zu; "
                    "launch %lld x %d threads, %d B dynamic smem\n",
-                   D, (int)CAUSAL, fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes,
+                   D, MASK, fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes,
                    fa.maxDynamicSharedSizeBytes, fa.localSizeBytes, grid, Cfg::THREADS, Cfg::SMEM_BYTES);
   }
   return e == cudaSuccess ? SDPA_OK : cuda_fail("prefill launch", e);
@@ -143,10 +145,37 @@ extern "C" int sdpa_fwd(const void* Q, const void* K, const void* V, void* O, fl
   if (int e = check_device()) return e;
   cudaStream_t s = (cudaStream_t)stream;
   if (d_k == 64)
-    return causal ? launch_prefill<64, true>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, s)
-                  : launch_prefill<64, false>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, s);
-  return causal ? launch_prefill<128, true>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, s)
-                : launch_prefill<128, false>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, s);
+    return causal ? launch_prefill<64, 1>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, -1, 0, s)
+                  : launch_prefill<64, 0>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, -1, -1, s);
+  return causal ? launch_prefill<128, 1>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, -1, 0, s)
+                : launch_prefill<128, 0>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, -1, -1, s);
+}
+
+extern "C" int sdpa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* LSE, int batch,
+                               int heads, int n_q, int n_kv, int d_k, int d_v, float scale, int window_left,
+                               int window_right, void* stream) {
+  if (batch < 0 || heads < 0 || n_q < 0 || n_kv < 1 || window_left < -1 || window_right < -1 || !std::isfinite(scale))
+    return SDPA_ERR_INVALID_ARG;
+  if (d_k != d_v || (d_k != 64 && d_k != 128) || !(scale > 0.f)) return SDPA_ERR_UNSUPPORTED;
+  if (batch == 0 || heads == 0 || n_q == 0) return SDPA_OK;
+  if (!Q || !K || !V || !O) return SDPA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (LSE && !aligned4(LSE)))
+    return SDPA_ERR_MISALIGNED;
+  const long long bh = (long long)batch * heads;
+  if (bh * (long long)(n_q > n_kv ? n_q : n_kv) >= (1LL << 31) || bh * ((n_q + 255) / 256) >= (1LL << 31))
+    return SDPA_ERR_UNSUPPORTED;
+  if (int e = check_device()) return e;
+  cudaStream_t s = (cudaStream_t)stream;
+  // Open windows are the plain kernels; everything else takes the windowed instantiation.
+  const int mode = window_left == -1 ? (window_right == -1 ? 0 : (window_right == 0 ? 1 : 2)) : 2;
+  if (d_k == 64) {
+    if (mode == 0) return launch_prefill<64, 0>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, -1, -1, s);
+    if (mode == 1) return launch_prefill<64, 1>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, -1, 0, s);
+    return launch_prefill<64, 2>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, window_left, window_right, s);
+  }
+  if (mode == 0) return launch_prefill<128, 0>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, -1, -1, s);
+  if (mode == 1) return launch_prefill<128, 1>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, -1, 0, s);
+  return launch_prefill<128, 2>(Q, K, V, O, LSE, (int)bh, n_q, n_kv, scale, window_left, window_right, s);
 }
 
 extern "C" int sdpa_fwd_f32(const float* Q, const float* K, const float* V, float* O, float* LSE, int batch,

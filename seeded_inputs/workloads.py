@@ -5,6 +5,7 @@
   cfg3  bf16 prefill, B=1 H=32 n=8192 d=128, Q,K ~ N(0,1), V ~ U(-1,1), scale 1/sqrt(128), causal
   cfg4  bf16 prefill, B=1 H=8 n=32768 d=128, Q,K ~ N(0, 2.5^2), V ~ N(0,1), scale 1/sqrt(128), non-causal
   cfg5  bf16 decode, B=64 H=32 n_cap=16384 d=128, lengths ~ U{1024..16384}, N(0,1), scale 1/sqrt(128)
+  cfg3w cfg3 with a causal local window of 512 keys (window_left = 511, window_right = 0)
 
 Streams: Q = 0, K = 1, V = 2 (counter = flat element index of the tensor), decode
 lengths = 3, sampled rows = 4.  Seed 0 everywhere.  bf16 values are the RNE
@@ -39,13 +40,25 @@ class Prefill:
     k: Dist = field(default_factory=Dist)
     v: Dist = field(default_factory=Dist)
     seed: int = 0
+    window: tuple = None  # (left, right) local window, -1 = open side; None = plain causal / full
 
     @property
     def scale_f32(self):
         return float(np.float32(self.scale))
 
+    def visible_pairs(self):
+        """Exact number of (query, key) pairs a window lets through, per (batch, head)."""
+        left, right = self.window
+        pos = np.arange(self.n_q, dtype=np.int64) + (self.n_kv - self.n_q)
+        hi = np.full_like(pos, self.n_kv - 1) if right < 0 else np.minimum(self.n_kv - 1, pos + right)
+        lo = np.zeros_like(pos) if left < 0 else np.maximum(0, pos - left)
+        return int(np.maximum(0, hi - lo + 1).sum())
+
     def flops(self):
-        """Algorithmic FLOPs: two matmuls at 2 FLOP per multiply-add, halved under a causal mask."""
+        """Algorithmic FLOPs: two matmuls at 2 FLOP per multiply-add, halved under a causal mask
+        (for a window: 4 d FLOP per visible (query, key) pair)."""
+        if self.window is not None:
+            return 4.0 * self.d * self.batch * self.heads * self.visible_pairs()
         f = 2.0 * self.batch * self.heads * self.n_q * self.n_kv * (2 * self.d)
         return f / 2 if self.causal else f
 
@@ -96,6 +109,9 @@ CFG2C = CFG2.with_causal(True)
 CFG3 = Prefill("cfg3", 1, 32, 8192, 8192, 128, True, "bf16", 1 / 128 ** 0.5, v=Dist(UNIFORM, -1.0, 1.0))
 CFG4 = Prefill("cfg4", 1, 8, 32768, 32768, 128, False, "bf16", 1 / 128 ** 0.5, q=Dist(NORMAL, 0.0, 2.5),
                k=Dist(NORMAL, 0.0, 2.5))
+# cfg3's shape with a causal local window of 512 keys (each row sees itself and the 511 before it)
+CFG3W = Prefill("cfg3w", 1, 32, 8192, 8192, 128, True, "bf16", 1 / 128 ** 0.5, v=Dist(UNIFORM, -1.0, 1.0),
+                window=(511, 0))
 CFG5 = Decode("cfg5", 64, 32, 16384, 128, 1024, 16384, 1 / 128 ** 0.5)
 
 

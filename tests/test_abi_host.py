@@ -29,6 +29,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
         "sdpa_decode", "sdpa_decode_noalloc", "sdpa_decode_workspace_size", "sdpa_fwd", "sdpa_fwd_f32",
+        "sdpa_fwd_window",
         "sdpa_get_last_device_error", "sdpa_status_string"])
 
 
@@ -74,6 +75,18 @@ def test_fwd_argument_errors(sdpa):
     assert fwd(sdpa, Q=None, K=None, V=None, O=None, nq=0) == sdpa.SDPA_OK
     assert fwd(sdpa, Q=None, K=None, V=None, O=None, b=0) == sdpa.SDPA_OK
     assert fwd(sdpa, Q=None, K=None, V=None, O=None, h=0) == sdpa.SDPA_OK
+
+
+def test_fwd_window_argument_errors(sdpa):
+    f = lambda **kw: sdpa.lib.sdpa_fwd_window(*[kw.get(n, d) for n, d in (
+        ("Q", P), ("K", P), ("V", P), ("O", P), ("LSE", None), ("b", 1), ("h", 1), ("nq", 64), ("nkv", 64), ("dk", 64),
+        ("dv", 64), ("scale", 0.125), ("wl", 16), ("wr", 0), ("st", None))])
+    assert f(wl=-2) == sdpa.SDPA_ERR_INVALID_ARG
+    assert f(wr=-3) == sdpa.SDPA_ERR_INVALID_ARG
+    assert f(Q=None) == sdpa.SDPA_ERR_INVALID_ARG
+    assert f(dk=96, dv=96) == sdpa.SDPA_ERR_UNSUPPORTED
+    assert f(V=P + 2) == sdpa.SDPA_ERR_MISALIGNED
+    assert f(Q=None, K=None, V=None, O=None, nq=0) == sdpa.SDPA_OK
 
 
 def test_fwd_f32_argument_errors(sdpa):

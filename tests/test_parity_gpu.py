@@ -162,6 +162,67 @@ def test_cfg4_long_sampled(sdpa, cuda_device):
     _sampled_prefill(sdpa, cuda_device, W.CFG4, 256)
 
 
+# ------------------------------------------------------------------------------------- local windows (bf16)
+WINDOW_CASES = [
+    # (B, H, n_q, n_kv, d, left, right)
+    (1, 2, 300, 300, 64, 0, 0), (1, 2, 300, 300, 64, 5, 0), (1, 2, 600, 600, 128, 127, 0),
+    (1, 2, 600, 600, 64, 128, 0), (1, 3, 1000, 1000, 128, 300, 0), (1, 2, 512, 512, 64, 64, 64),
+    (1, 2, 400, 400, 128, -1, 5), (1, 2, 400, 400, 64, 200, -1), (1, 2, 257, 513, 128, 100, 0),
+    (1, 2, 513, 257, 64, 100, 0), (2, 2, 384, 384, 128, -1, 0), (1, 2, 384, 384, 64, -1, -1),
+    (1, 1, 700, 700, 64, 255, 255), (1, 2, 384, 384, 64, 5000, 0), (1, 2, 384, 512, 128, 5000, 5000),
+]
+
+
+@pytest.mark.parametrize("B,H,n_q,n_kv,d,left,right", WINDOW_CASES)
+def test_prefill_window_small(sdpa, cuda_device, B, H, n_q, n_kv, d, left, right):
+    import torch
+    seed = 1000 + n_q + 7 * n_kv + 13 * d + left
+    q = si.fill_host((B, H, n_q, d), seed, 0)
+    k = si.fill_host((B, H, n_kv, d), seed, 1)
+    v = si.fill_host((B, H, n_kv, d), seed, 2)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    _, tq = _bits_to_torch(q, cuda_device, 128 * d)
+    _, tk = _bits_to_torch(k, cuda_device, 128 * d)
+    _, tv = _bits_to_torch(v, cuda_device, 128 * d)
+    o_flat, o = _nan_buffer((B, H, n_q, d), torch.bfloat16, cuda_device, 128 * d)
+    l_flat, lse = _nan_buffer((B, H, n_q), torch.float32, cuda_device, 256)
+    sdpa.fwd_window(tq, tk, tv, left, right, scale=scale, o=o, lse=lse)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O_ref, L_ref = oracle.sdpa_rows_window(*(si.bf16_bits_to_f32(x) for x in (q, k, v)), scale, left, right)
+    check_bf16(o.float().cpu().numpy(), O_ref, lse.cpu().numpy(), L_ref, "window %s" % ((B, H, n_q, n_kv, d, left, right),))
+    assert torch.isnan(o_flat[o.numel():]).all() and torch.isnan(l_flat[lse.numel():]).all()
+
+
+def test_window_open_sides_equal_plain_calls(sdpa, cuda_device):
+    import torch
+    B, H, n, d = 1, 2, 640, 128
+    q, k, v = (W.to_torch(si.fill_host((B, H, n, d), 9, s_), cuda_device) for s_ in (0, 1, 2))
+    for causal, (left, right) in ((False, (-1, -1)), (True, (-1, 0))):
+        o1, l1 = sdpa.fwd(q, k, v, causal=causal)
+        o2, l2 = sdpa.fwd_window(q, k, v, left, right)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_cfg3w_window_full_size_sampled(sdpa, cuda_device):
+    import torch
+    w = W.CFG3W
+    host = W.prefill_host(w)
+    tq, tk, tv = (W.to_torch(host[n], cuda_device) for n in ("q", "k", "v"))
+    o, lse = sdpa.fwd_window(tq, tk, tv, w.window[0], w.window[1], scale=w.scale_f32)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O = o.float().cpu().numpy()
+    L = lse.cpu().numpy()
+    del tq, tk, tv, o, lse
+    torch.cuda.empty_cache()
+    qf, kf, vf = (W.as_f32(host[n]) for n in ("q", "k", "v"))
+    for h in range(0, w.heads, 4):
+        rows = si.sample_rows(w.n_q, 128, w.seed, salt=h)
+        O_ref, L_ref = oracle.sdpa_rows_window(qf[0, h], kf[0, h], vf[0, h], w.scale_f32, w.window[0], w.window[1],
+                                               rows=rows)
+        check_bf16(O[0, h, rows], O_ref, L[0, h, rows], L_ref, "cfg3w h=%d" % h)
+
+
 # ----------------------------------------------------------------------------------------------- fp32 path
 F32_CASES = [(1, 1, 128, 128, 64, 64, False), (1, 1, 128, 128, 64, 64, True), (2, 3, 77, 130, 33, 100, True),
              (1, 2, 200, 50, 128, 128, True), (1, 1, 1, 1, 1, 1, False), (1, 2, 65, 300, 3, 128, False)]
