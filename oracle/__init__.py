@@ -45,6 +45,9 @@ def lib():
         L.oracle_sdpa_rows_window.restype = ctypes.c_int
         L.oracle_decode.argtypes = [_f32p, _f32p, _f32p, _i32p, I64, I64, I64, I32, I32, D, _i64p, I64,
                                     _f64p, _f64p, I32]
+        L.oracle_decode_gqa.argtypes = [_f32p, _f32p, _f32p, _i32p, I64, I64, I64, I64, I32, I32, D, _i64p, I64,
+                                        _f64p, _f64p, I32]
+        L.oracle_decode_gqa.restype = ctypes.c_int
         for f in (L.oracle_scores, L.oracle_softmax_rows, L.oracle_softmax_naive, L.oracle_sdpa_full,
                   L.oracle_sdpa_rows, L.oracle_decode):
             f.restype = ctypes.c_int
@@ -168,4 +171,26 @@ def decode(q, k, v, lens, scale, pairs=None, threads=None):
     _check(lib().oracle_decode(qp, kp, vp, lens.ctypes.data_as(_i32p), B, H, n_cap, d_k, d_v, scale, pp,
                                n_pairs, O.ctypes.data_as(_f64p), L.ctypes.data_as(_f64p),
                                threads or threads_available()), "oracle_decode")
+    return O, L
+
+
+def decode_gqa(q, k, v, lens, scale, pairs=None, threads=None):
+    """Grouped-query decode. q [B, H_q, d_k], k/v [B, H_kv, n_cap, d], lens [B]; query head h reads
+    key/value head h // (H_q // H_kv).  Returns O [n_pairs, d_v], LSE [n_pairs] (pairs = b*H_q + h)."""
+    B, H_kv, n_cap, d_k = k.shape
+    H_q = q.shape[1]
+    d_v = v.shape[-1]
+    q, qp = _f32(q)
+    k, kp = _f32(k)
+    v, vp = _f32(v)
+    lens = np.ascontiguousarray(lens, dtype=np.int32)
+    if pairs is None:
+        pp, n_pairs = None, B * H_q
+    else:
+        pairs = np.ascontiguousarray(pairs, dtype=np.int64)
+        pp, n_pairs = pairs.ctypes.data_as(_i64p), pairs.shape[0]
+    O = np.empty((n_pairs, d_v)); L = np.empty((n_pairs,))
+    _check(lib().oracle_decode_gqa(qp, kp, vp, lens.ctypes.data_as(_i32p), B, H_q, H_kv, n_cap, d_k, d_v, scale,
+                                   pp, n_pairs, O.ctypes.data_as(_f64p), L.ctypes.data_as(_f64p),
+                                   threads or threads_available()), "oracle_decode_gqa")
     return O, L

@@ -225,3 +225,28 @@ extern "C" int oracle_sdpa_rows_window(const float* Q, const float* K, const flo
   });
   return 0;
 }
+
+extern "C" int oracle_decode_gqa(const float* Q, const float* K, const float* V, const int32_t* lens, int64_t B,
+                                 int64_t H_q, int64_t H_kv, int64_t n_cap, int d_k, int d_v, double scale,
+                                 const int64_t* pairs, int64_t n_pairs, double* O, double* LSE, int threads) {
+  if (B < 0 || H_q < 0 || H_kv <= 0 || n_cap <= 0 || d_k <= 0 || d_v <= 0) return -1;
+  if (H_q % H_kv != 0) return -1;
+  if (!pairs) n_pairs = B * H_q;
+  if (n_pairs <= 0) return 0;
+  if (!Q || !K || !V || !lens || !O || !LSE) return -1;
+  for (int64_t b = 0; b < B; ++b)
+    if (lens[b] < 1 || lens[b] > n_cap) return -1;
+  for (int64_t p = 0; pairs && p < n_pairs; ++p)
+    if (pairs[p] < 0 || pairs[p] >= B * H_q) return -1;
+  const int64_t group = H_q / H_kv;  // query heads per key/value head
+  parallel_for(n_pairs, threads, [&](int64_t p) {
+    const int64_t bh = pairs ? pairs[p] : p;
+    const int64_t b = bh / H_q, h = bh % H_q;
+    const int64_t kv = b * H_kv + h / group;  // the key/value head this query head reads
+    const int64_t n = lens[b];
+    std::vector<double> s((size_t)n);
+    score_row(Q + bh * d_k, K + kv * n_cap * d_k, 0, 1, n, d_k, scale, 0, s.data());
+    attend_row(s.data(), V + kv * n_cap * d_v, n, d_v, O + p * d_v, LSE + p);
+  });
+  return 0;
+}

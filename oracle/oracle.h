@@ -27,6 +27,11 @@
  * slices back to back ([bh, n, d]).  Inputs are float32: every bf16 and fp32
  * input value is exact in float32 and is widened exactly to double here.
  *
+ * Grouped-query decode (several query heads reading one key/value head) is the
+ * same definition with the key/value head chosen by the query head's group; the
+ * 2-simplicial article (szyisi.cn, "model design") tiles along the query heads
+ * of such groups to keep its kernels dense.
+ *
  * Parity pins: see tests/test_oracle_pins.py (closed forms, invariants, brute
  * force, a hand-worked example and a library special case).
  */
@@ -79,6 +84,15 @@ int oracle_sdpa_rows_window(const float* Q, const float* K, const float* V, int6
 int oracle_decode(const float* Q, const float* K, const float* V, const int32_t* lens, int64_t B,
                   int64_t H, int64_t n_cap, int d_k, int d_v, double scale, const int64_t* pairs,
                   int64_t n_pairs, double* O, double* LSE, int threads);
+
+/* Grouped-query decode: H_q query heads share H_kv key/value heads (H_q a multiple of H_kv),
+   query head h reading key/value head h / (H_q / H_kv) -- consecutive query heads form a group.
+   Q [B, H_q, d_k]; K [B, H_kv, n_cap, d_k]; V [B, H_kv, n_cap, d_v]; O [B, H_q, d_v]; LSE [B, H_q].
+   pairs: flat b*H_q + h indices as in oracle_decode (NULL = all, in order).  H_kv == H_q is
+   oracle_decode. */
+int oracle_decode_gqa(const float* Q, const float* K, const float* V, const int32_t* lens, int64_t B,
+                      int64_t H_q, int64_t H_kv, int64_t n_cap, int d_k, int d_v, double scale,
+                      const int64_t* pairs, int64_t n_pairs, double* O, double* LSE, int threads);
 
 #ifdef __cplusplus
 }

@@ -25,6 +25,8 @@ MUTANTS = {
     "window_left_off_by_one": ("if (left >= 0 && j < pos - left) return false;", "if (left >= 0 && j <= pos - left) return false;"),
     "window_right_ignored": ("if (right >= 0 && j > pos + right) return false;", ""),
     "window_position_top_left": ("const int64_t pos = i + (n_kv - n_q);", "const int64_t pos = i;"),
+    "gqa_heads_interleaved": ("const int64_t kv = b * H_kv + h / group;", "const int64_t kv = b * H_kv + h % H_kv;"),
+    "gqa_v_head_interleaved": ("attend_row(s.data(), V + kv * n_cap * d_v,", "attend_row(s.data(), V + (b * H_kv + h % H_kv) * n_cap * d_v,"),
 }
 
 

@@ -325,3 +325,70 @@ def test_window_brute_force(n_q, n_kv, left, right):
     assert (np.isneginf(L) == np.isneginf(Lb)).all()
     fin = np.isfinite(Lb)
     np.testing.assert_allclose(L[fin], Lb[fin], rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------------------------------------------ grouped-query decode
+# Query head h of H_q reads key/value head h // (H_q // H_kv): consecutive query heads share one
+# key/value head (the grouped-query layout the 2-simplicial article tiles along).
+def test_gqa_equals_decode_on_an_expanded_cache():
+    # Replicating every key/value head over its group turns grouped-query decode into plain decode.
+    B, H_q, H_kv, n_cap, d = 3, 8, 2, 11, 5
+    q = RNG.standard_normal((B, H_q, d)).astype(np.float32)
+    k = RNG.standard_normal((B, H_kv, n_cap, d)).astype(np.float32)
+    v = RNG.standard_normal((B, H_kv, n_cap, 4)).astype(np.float32)
+    lens = np.array([11, 1, 6], np.int32)
+    G = H_q // H_kv
+    k_exp = np.repeat(k, G, axis=1)  # head h of the expanded cache is head h // G
+    v_exp = np.repeat(v, G, axis=1)
+    O, L = oracle.decode_gqa(q, k, v, lens, 0.7)
+    Oe, Le = oracle.decode(q, k_exp, v_exp, lens, 0.7)
+    np.testing.assert_array_equal(O, Oe)
+    np.testing.assert_array_equal(L, Le)
+
+
+def test_gqa_group_of_one_is_decode_and_pairs_select():
+    B, H, n_cap, d = 2, 3, 7, 4
+    q = RNG.standard_normal((B, H, d)).astype(np.float32)
+    k = RNG.standard_normal((B, H, n_cap, d)).astype(np.float32)
+    v = RNG.standard_normal((B, H, n_cap, d)).astype(np.float32)
+    lens = np.array([7, 3], np.int32)
+    O, L = oracle.decode_gqa(q, k, v, lens, 0.5)
+    Od, Ld = oracle.decode(q, k, v, lens, 0.5)
+    np.testing.assert_array_equal(O, Od)
+    np.testing.assert_array_equal(L, Ld)
+    pairs = np.array([5, 0, 3], np.int64)
+    Op, Lp = oracle.decode_gqa(q, k, v, lens, 0.5, pairs=pairs)
+    np.testing.assert_array_equal(Op, O[pairs])
+    np.testing.assert_array_equal(Lp, L[pairs])
+
+
+def test_gqa_brute_force_and_group_closed_form():
+    # Brute force in plain Python; and a group whose queries are all zero attends uniformly:
+    # O = mean of the first len rows of its key/value head's V, LSE = ln len.
+    B, H_q, H_kv, n_cap, d = 2, 6, 3, 5, 3
+    q = RNG.uniform(-1, 1, (B, H_q, d)).astype(np.float32)
+    q[1, 2:4] = 0.0  # batch 1, group 1 (query heads 2 and 3 -> key/value head 1)
+    k = RNG.uniform(-1, 1, (B, H_kv, n_cap, d)).astype(np.float32)
+    v = RNG.standard_normal((B, H_kv, n_cap, 2)).astype(np.float32)
+    lens = np.array([5, 4], np.int32)
+    O, L = oracle.decode_gqa(q, k, v, lens, 1.3)
+    G = H_q // H_kv
+    for b in range(B):
+        for h in range(H_q):
+            kv = h // G
+            n = int(lens[b])
+            w = [math.exp(1.3 * math.fsum(float(a) * float(c) for a, c in zip(q[b, h], k[b, kv, j])))
+                 for j in range(n)]
+            z = math.fsum(w)
+            ref = [math.fsum(w[j] * float(v[b, kv, j, c]) for j in range(n)) / z for c in range(2)]
+            np.testing.assert_allclose(O[b * H_q + h], ref, rtol=1e-13, atol=1e-14)
+            assert abs(L[b * H_q + h] - math.log(z)) < 1e-13
+    for h in (2, 3):
+        np.testing.assert_allclose(O[1 * H_q + h], v[1, 1, :4].astype(np.float64).mean(axis=0), rtol=1e-14)
+        assert abs(L[1 * H_q + h] - math.log(4)) < 1e-14
+
+
+def test_gqa_rejects_bad_groups():
+    with pytest.raises(ValueError):
+        oracle.decode_gqa(np.zeros((1, 3, 4), np.float32), np.zeros((1, 2, 4, 4), np.float32),
+                          np.zeros((1, 2, 4, 4), np.float32), np.array([4], np.int32), 1.0)
