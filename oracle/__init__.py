@@ -48,6 +48,9 @@ def lib():
         L.oracle_decode_gqa.argtypes = [_f32p, _f32p, _f32p, _i32p, I64, I64, I64, I64, I32, I32, D, _i64p, I64,
                                         _f64p, _f64p, I32]
         L.oracle_decode_gqa.restype = ctypes.c_int
+        L.oracle_sdpa_backward.argtypes = [_f32p, _f32p, _f32p, _f32p, I64, I64, I64, I32, I32, D, I32, _i64p, I64,
+                                           _i64p, I64, _f64p, _f64p, _f64p, I32]
+        L.oracle_sdpa_backward.restype = ctypes.c_int
         for f in (L.oracle_scores, L.oracle_softmax_rows, L.oracle_softmax_naive, L.oracle_sdpa_full,
                   L.oracle_sdpa_rows, L.oracle_decode):
             f.restype = ctypes.c_int
@@ -194,3 +197,36 @@ def decode_gqa(q, k, v, lens, scale, pairs=None, threads=None):
                                    pp, n_pairs, O.ctypes.data_as(_f64p), L.ctypes.data_as(_f64p),
                                    threads or threads_available()), "oracle_decode_gqa")
     return O, L
+
+
+def sdpa_backward(q, k, v, do, scale, causal=False, q_rows=None, k_rows=None, threads=None):
+    """Gradients of exact attention for loss gradient `do`, over leading slice dims.
+
+    q [..., n_q, d_k], k [..., n_kv, d_k], v [..., n_kv, d_v], do [..., n_q, d_v].
+    q_rows / k_rows: None (all) or 1-D index arrays applied to every slice.
+    Returns dQ [..., n_qr, d_k], dK [..., n_kr, d_k], dV [..., n_kr, d_v] in float64.
+    """
+    lead = q.shape[:-2]
+    n_q, d_k = q.shape[-2:]
+    n_kv, d_v = v.shape[-2:]
+    bh = int(np.prod(lead, dtype=np.int64)) if lead else 1
+    q, qp = _f32(q)
+    k, kp = _f32(k)
+    v, vp = _f32(v)
+    do, dop = _f32(do)
+    if q_rows is None:
+        qrp, n_qr = None, n_q
+    else:
+        q_rows = np.ascontiguousarray(q_rows, dtype=np.int64)
+        qrp, n_qr = q_rows.ctypes.data_as(_i64p), q_rows.shape[0]
+    if k_rows is None:
+        krp, n_kr = None, n_kv
+    else:
+        k_rows = np.ascontiguousarray(k_rows, dtype=np.int64)
+        krp, n_kr = k_rows.ctypes.data_as(_i64p), k_rows.shape[0]
+    dQ = np.empty(lead + (n_qr, d_k)); dK = np.empty(lead + (n_kr, d_k)); dV = np.empty(lead + (n_kr, d_v))
+    _check(lib().oracle_sdpa_backward(qp, kp, vp, dop, bh, n_q, n_kv, d_k, d_v, scale, int(causal), qrp, n_qr, krp,
+                                      n_kr, dQ.ctypes.data_as(_f64p), dK.ctypes.data_as(_f64p),
+                                      dV.ctypes.data_as(_f64p), threads or threads_available()),
+           "oracle_sdpa_backward")
+    return dQ, dK, dV

@@ -250,3 +250,75 @@ extern "C" int oracle_decode_gqa(const float* Q, const float* K, const float* V,
   });
   return 0;
 }
+
+extern "C" int oracle_sdpa_backward(const float* Q, const float* K, const float* V, const float* dO, int64_t bh,
+                                    int64_t n_q, int64_t n_kv, int d_k, int d_v, double scale, int causal,
+                                    const int64_t* q_rows, int64_t n_qr, const int64_t* k_rows, int64_t n_kr,
+                                    double* dQ, double* dK, double* dV, int threads) {
+  if (bh < 0 || n_q < 0 || n_kv <= 0 || d_k <= 0 || d_v <= 0) return -1;
+  if (!q_rows) n_qr = n_q;
+  if (!k_rows) n_kr = n_kv;
+  if (n_qr < 0 || n_kr < 0) return -1;
+  if (bh == 0 || n_q == 0) return 0;
+  if (!Q || !K || !V || !dO) return -1;
+  for (int64_t r = 0; q_rows && r < n_qr; ++r)
+    if (q_rows[r] < 0 || q_rows[r] >= n_q) return -1;
+  for (int64_t r = 0; k_rows && r < n_kr; ++r)
+    if (k_rows[r] < 0 || k_rows[r] >= n_kv) return -1;
+  // where each query / key row lands in the outputs (-1: not requested)
+  std::vector<int64_t> q_slot((size_t)n_q, -1), k_slot((size_t)n_kv, -1);
+  for (int64_t r = 0; r < n_qr; ++r) q_slot[(size_t)(q_rows ? q_rows[r] : r)] = r;
+  for (int64_t r = 0; r < n_kr; ++r) k_slot[(size_t)(k_rows ? k_rows[r] : r)] = r;
+  parallel_for(bh, threads, [&](int64_t b) {
+    const float* Qb = Q + b * n_q * d_k;
+    const float* Kb = K + b * n_kv * d_k;
+    const float* Vb = V + b * n_kv * d_v;
+    const float* dOb = dO + b * n_q * d_v;
+    double* dQb = dQ ? dQ + b * n_qr * d_k : nullptr;
+    double* dKb = dK ? dK + b * n_kr * d_k : nullptr;
+    double* dVb = dV ? dV + b * n_kr * d_v : nullptr;
+    if (dQb)
+      for (int64_t t = 0; t < n_qr * d_k; ++t) dQb[t] = 0.0;
+    if (dKb)
+      for (int64_t t = 0; t < n_kr * d_k; ++t) dKb[t] = 0.0;
+    if (dVb)
+      for (int64_t t = 0; t < n_kr * d_v; ++t) dVb[t] = 0.0;
+    std::vector<double> s((size_t)n_kv), p((size_t)n_kv), dp((size_t)n_kv);
+    for (int64_t i = 0; i < n_q; ++i) {
+      // row i of P = softmax(S): the forward definition
+      score_row(Qb, Kb, i, n_q, n_kv, d_k, scale, causal, s.data());
+      double m, l;
+      softmax_row(s.data(), n_kv, p.data(), &m, &l);
+      if (m == kNegInf) continue;  // no allowed key: no gradient flows through this row
+      // row i of dP = dO V^T, and the softmax Jacobian's row term sum_k P_ik dP_ik
+      const float* dOi = dOb + i * d_v;
+      double rowdot = 0.0;
+      for (int64_t j = 0; j < n_kv; ++j) {
+        double acc = 0.0;
+        const float* vj = Vb + j * d_v;
+        for (int c = 0; c < d_v; ++c) acc += (double)dOi[c] * (double)vj[c];
+        dp[(size_t)j] = acc;
+        rowdot += p[(size_t)j] * acc;
+      }
+      const int64_t qi = q_slot[(size_t)i];
+      for (int64_t j = 0; j < n_kv; ++j) {
+        const double pij = p[(size_t)j];
+        if (pij == 0.0) continue;
+        const double dsij = pij * (dp[(size_t)j] - rowdot);
+        if (dQb && qi >= 0) {  // dQ_i += scale dS_ij K_j
+          const float* kj = Kb + j * d_k;
+          for (int c = 0; c < d_k; ++c) dQb[qi * d_k + c] += scale * dsij * (double)kj[c];
+        }
+        const int64_t kj_slot = k_slot[(size_t)j];
+        if (kj_slot < 0) continue;
+        if (dVb)  // dV_j += P_ij dO_i
+          for (int c = 0; c < d_v; ++c) dVb[kj_slot * d_v + c] += pij * (double)dOi[c];
+        if (dKb) {  // dK_j += scale dS_ij Q_i
+          const float* qi_row = Qb + i * d_k;
+          for (int c = 0; c < d_k; ++c) dKb[kj_slot * d_k + c] += scale * dsij * (double)qi_row[c];
+        }
+      }
+    }
+  });
+  return 0;
+}

@@ -32,6 +32,11 @@
  * 2-simplicial article (szyisi.cn, "model design") tiles along the query heads
  * of such groups to keep its kernels dense.
  *
+ * The backward pass is the chain rule through the same definition: the
+ * MoA roadmap's last stage is a DNF for the backward pass (agents-report.net MoA
+ * article, "implementation roadmap"); its result is the ordinary gradient of exact
+ * attention.
+ *
  * Parity pins: see tests/test_oracle_pins.py (closed forms, invariants, brute
  * force, a hand-worked example and a library special case).
  */
@@ -93,6 +98,20 @@ int oracle_decode(const float* Q, const float* K, const float* V, const int32_t*
 int oracle_decode_gqa(const float* Q, const float* K, const float* V, const int32_t* lens, int64_t B,
                       int64_t H_q, int64_t H_kv, int64_t n_cap, int d_k, int d_v, double scale,
                       const int64_t* pairs, int64_t n_pairs, double* O, double* LSE, int threads);
+
+/* Backward pass of one (batch, head) slice at a time, for the forward above (causal or not).
+   With P = softmax_rows(S) and loss gradient dO = dL/dO:
+     dV = P^T dO;  dP = dO V^T;  dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik);
+     dQ = scale dS K;  dK = scale dS^T Q.
+   Every query row is visited (each row's softmax is needed for every key column); only the
+   listed outputs are written: dQ rows q_rows (n_qr of them, NULL = all n_q in order) into
+   dQ [bh, n_qr, d_k]; dK and dV rows k_rows (NULL = all n_kv) into dK [bh, n_kr, d_k] and
+   dV [bh, n_kr, d_v].  Output pointers may be NULL to skip that output.  A row with no
+   allowed key contributes nothing.  threads <= 0 means 1. */
+int oracle_sdpa_backward(const float* Q, const float* K, const float* V, const float* dO, int64_t bh,
+                         int64_t n_q, int64_t n_kv, int d_k, int d_v, double scale, int causal,
+                         const int64_t* q_rows, int64_t n_qr, const int64_t* k_rows, int64_t n_kr, double* dQ,
+                         double* dK, double* dV, int threads);
 
 #ifdef __cplusplus
 }

@@ -26,6 +26,9 @@ MUTANTS = {
     "window_right_ignored": ("if (right >= 0 && j > pos + right) return false;", ""),
     "window_position_top_left": ("const int64_t pos = i + (n_kv - n_q);", "const int64_t pos = i;"),
     "gqa_heads_interleaved": ("const int64_t kv = b * H_kv + h / group;", "const int64_t kv = b * H_kv + h % H_kv;"),
+    "bwd_drops_jacobian_row_term": ("const double dsij = pij * (dp[(size_t)j] - rowdot);", "const double dsij = pij * dp[(size_t)j];"),
+    "bwd_dk_without_scale": ("dKb[kj_slot * d_k + c] += scale * dsij * (double)qi_row[c];", "dKb[kj_slot * d_k + c] += dsij * (double)qi_row[c];"),
+    "bwd_dv_uses_transposed_index": ("dVb[kj_slot * d_v + c] += pij * (double)dOi[c];", "dVb[kj_slot * d_v + c] += pij * (double)dOb[(n_q - 1 - i) * d_v + c];"),
     "gqa_v_head_interleaved": ("attend_row(s.data(), V + kv * n_cap * d_v,", "attend_row(s.data(), V + (b * H_kv + h % H_kv) * n_cap * d_v,"),
 }
 

@@ -392,3 +392,93 @@ def test_gqa_rejects_bad_groups():
     with pytest.raises(ValueError):
         oracle.decode_gqa(np.zeros((1, 3, 4), np.float32), np.zeros((1, 2, 4, 4), np.float32),
                           np.zeros((1, 2, 4, 4), np.float32), np.array([4], np.int32), 1.0)
+
+
+# ------------------------------------------------------------------------------------------- backward pass
+# The gradients of L = sum(O * dO) for the forward definition (the MoA roadmap's last stage is
+# the backward pass).  Pinned by finite differences of the forward oracle, torch float64
+# autograd, and identities that hold for any inputs.
+def _loss(q, k, v, do, scale, causal):
+    O, _ = oracle.sdpa_rows(q, k, v, scale, causal)
+    return float(np.sum(O * do.astype(np.float64)))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_finite_differences(causal):
+    n_q, n_kv, d_k, d_v = 4, 6, 3, 2
+    g = np.random.default_rng(7)
+    # dyadic inputs well inside float32: perturbations of +-2^-12 are exact
+    q = (g.integers(-8, 9, (n_q, d_k)) / 8).astype(np.float32)
+    k = (g.integers(-8, 9, (n_kv, d_k)) / 8).astype(np.float32)
+    v = (g.integers(-8, 9, (n_kv, d_v)) / 8).astype(np.float32)
+    do = (g.integers(-8, 9, (n_q, d_v)) / 8).astype(np.float32)
+    scale, h = 0.7, 2.0 ** -12
+    dQ, dK, dV = oracle.sdpa_backward(q, k, v, do, scale, causal)
+    for x, grad in ((q, dQ), (k, dK), (v, dV)):
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [xp if y is x else y for y in (q, k, v)]
+            args_m = [xm if y is x else y for y in (q, k, v)]
+            fd = (_loss(*args_p, do, scale, causal) - _loss(*args_m, do, scale, causal)) / (2 * h)
+            assert abs(fd - grad[idx]) < 1e-7, (idx, fd, grad[idx])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_torch_float64_autograd(causal):
+    import torch
+    B, H, n_q, n_kv, d = 2, 2, 9, 13, 8
+    g = np.random.default_rng(8)
+    q, k, v, do = (g.standard_normal(s).astype(np.float32) for s in
+                   ((B, H, n_q, d), (B, H, n_kv, d), (B, H, n_kv, d), (B, H, n_q, d)))
+    scale = 0.3
+    dQ, dK, dV = oracle.sdpa_backward(q, k, v, do, scale, causal)
+    tq, tk, tv = (torch.from_numpy(x).double().requires_grad_(True) for x in (q, k, v))
+    # bottom-right aligned causal mask written out: row i sees keys j <= i + n_kv - n_q
+    mask = None
+    if causal:
+        mask = torch.from_numpy(np.arange(n_kv)[None, :] <= np.arange(n_q)[:, None] + (n_kv - n_q))
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=scale)
+    out.backward(torch.from_numpy(do).double())
+    np.testing.assert_allclose(dQ, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dK, tk.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dV, tv.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_identities(causal):
+    # Rows of P sum to one: sum_j dV_j = sum_i dO_i (over rows that see a key).  Rows of dS sum
+    # to zero: sum_j dK_j = 0.  Adding a constant row to V leaves dQ and dK unchanged.
+    n_q, n_kv, d = 11, 7, 5
+    q, k, do = (RNG.standard_normal(s).astype(np.float32) for s in ((n_q, d), (n_kv, d), (n_q, d)))
+    v = (RNG.integers(-64, 65, (n_kv, d)) / 16).astype(np.float32)  # dyadic: v + 3 is exact
+    dQ, dK, dV = oracle.sdpa_backward(q, k, v, do, 0.45, causal)
+    seen = np.arange(n_q) + (n_kv - n_q) >= 0 if causal else np.ones(n_q, bool)
+    np.testing.assert_allclose(dV.sum(axis=0), do[seen].astype(np.float64).sum(axis=0), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dK.sum(axis=0), 0.0, atol=1e-12)
+    dQ2, dK2, _ = oracle.sdpa_backward(q, k, v + np.float32(3.0), do, 0.45, causal)
+    np.testing.assert_allclose(dQ2, dQ, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dK2, dK, rtol=1e-10, atol=1e-12)
+
+
+def test_backward_single_key_closed_form():
+    # One key: P = 1 everywhere, so dV_0 = sum_i dO_i and dQ = dK = 0 exactly.
+    q = RNG.standard_normal((5, 4)).astype(np.float32)
+    k = RNG.standard_normal((1, 4)).astype(np.float32)
+    v = RNG.standard_normal((1, 3)).astype(np.float32)
+    do = RNG.standard_normal((5, 3)).astype(np.float32)
+    dQ, dK, dV = oracle.sdpa_backward(q, k, v, do, 0.9)
+    assert (dQ == 0).all() and (dK == 0).all()
+    np.testing.assert_allclose(dV[0], do.astype(np.float64).sum(axis=0), rtol=1e-15)
+
+
+def test_backward_row_selection():
+    n_q, n_kv, d = 10, 12, 4
+    q, k, v, do = (RNG.standard_normal(s).astype(np.float32) for s in ((n_q, d), (n_kv, d), (n_kv, d), (n_q, d)))
+    dQ, dK, dV = oracle.sdpa_backward(q, k, v, do, 0.5, True)
+    qr, kr = np.array([9, 0, 4]), np.array([11, 3])
+    sQ, sK, sV = oracle.sdpa_backward(q, k, v, do, 0.5, True, q_rows=qr, k_rows=kr)
+    np.testing.assert_array_equal(sQ, dQ[qr])
+    np.testing.assert_array_equal(sK, dK[kr])
+    np.testing.assert_array_equal(sV, dV[kr])
