@@ -40,6 +40,8 @@ sys.path.insert(0, ROOT)
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_SOURCES = ["memory_optimal_sdpa_b200/csrc/prefill_bf16.cuh", "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
 DECODE_SOURCES = ["memory_optimal_sdpa_b200/csrc/decode.cuh"]
+GQA_SOURCES = ["memory_optimal_sdpa_b200/csrc/decode_gqa.cuh", "memory_optimal_sdpa_b200/csrc/decode.cuh",
+               "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
 
 
 def load_peaks():
@@ -200,6 +202,30 @@ def oracle_rate(w_list, seconds_target, seed=0):
 
 
 # --------------------------------------------------------------------------------------------------- our arm
+def cost_model(flops, nbytes, t_meas, peaks, standard_bytes=None):
+    """The pages' execution-time model T = alpha F + beta M (MoA article, "memory bottleneck"), alpha and
+    beta the reciprocals of this GPU's measured dense bf16 rate and HBM copy bandwidth, against the
+    measured time; with the traffic of an implementation that writes and reads the score and
+    probability matrices, the speedup the model predicts for avoiding them."""
+    a = 1.0 / (peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]) * 1e12)
+    b = 1.0 / (peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]) * 1e9)
+    t_add = a * flops + b * nbytes
+    out = {"alpha_s_per_flop": a, "beta_s_per_byte": b, "flop": float(flops), "bytes": float(nbytes),
+           "predicted_ms": round(t_add * 1e3, 5), "roofline_ms": round(max(a * flops, b * nbytes) * 1e3, 5),
+           "measured_ms": round(t_meas * 1e3, 5), "measured_over_predicted": round(t_meas / t_add, 3)}
+    if standard_bytes is not None:
+        t_std = a * flops + b * standard_bytes
+        out.update({"standard_bytes": float(standard_bytes), "standard_predicted_ms": round(t_std * 1e3, 5),
+                    "predicted_speedup_vs_standard": round(t_std / t_add, 2)})
+    return out
+
+
+def standard_bytes(w):
+    """Traffic of the textbook implementation: the DNF's bytes plus the score matrix written and read
+    in fp32 and the probabilities written and read in bf16 (12 bytes per query-key pair, every pair)."""
+    return w.bytes() + w.batch * w.heads * w.n_q * w.n_kv * 12
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -319,8 +345,14 @@ def run_ours(args):
            "d2h_bytes_per_step": d2h}
     del hq, hk, hv, ho, dq, dk, dv
 
+    # ---- backward pass on the same workload (its own sub-benchmark)
+    backward = None if args.skip_backward else run_backward(args, sdpa, si, W, works, q, k, v, outs, stream, flush,
+                                                             peaks, peak_kind)
+
     # ---- decode workload (HBM-bound), its own roofline
     decode = None if args.skip_decode else run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind)
+    decode_gqa = (None if args.skip_decode else
+                  run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, grouped=True))
 
     line = {
         "metric": "attention fwd TFLOP/s (prefill) & decode HBM GB/s, as % of B200 roofline",
@@ -333,12 +365,18 @@ def run_ours(args):
                    "parallelism": "replicas x%d (independent heads, no collective)" % world,
                    "l2": "flushed before every timed step (256 MiB write, not timed)"},
         "roofline": roof,
+        "cost_model": {w.name: cost_model(w.flops(), w.bytes(), float(per_launch[:, i].mean()), peaks, standard_bytes(w))
+                       for i, w in enumerate(works)},
         "gpu_launches": args.steps * len(works),
         "e2e": e2e,
         "clocks": clocks.summary(t_wall0, t_wall1),
     }
+    if backward is not None:
+        line["backward"] = backward
     if decode is not None:
         line["decode"] = decode
+    if decode_gqa is not None:
+        line["decode_gqa"] = decode_gqa
     if rank == 0 and world == 1 and not args.skip_cpu:
         rate, cores, desc, secs = oracle_rate(works, args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(rate, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
@@ -350,15 +388,59 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind):
+def run_backward(args, sdpa, si, W, works, q, k, v, outs, stream, flush, peaks, peak_kind):
+    """dQ, dK, dV of each prefill workload of the step, from the forward's O and LSE.  Algorithmic
+    FLOPs: 2.5x the forward's (five matrix products of the gradient); the kernels execute seven
+    (S and dP are formed in both the dK/dV and the dQ kernel)."""
     import torch
-    w = W.CFG5
+    w0 = works[0]
+    do = W.to_torch(si.fill_host((w0.batch, w0.heads, w0.n_q, w0.d), w0.seed, si.STREAM_DO), q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(sdpa.bwd_workspace_size(w0.batch, w0.heads, w0.n_q), dtype=torch.uint8, device=q.device)
+    res = {}
+    for w, (o, lse) in zip(works, outs):
+        if w.window is not None:  # the backward pass takes full or causal attention
+            continue
+        call = lambda: sdpa.bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale_f32, dq=dq, dk=dk, dv=dv,
+                                workspace=ws, stream=stream)
+        for _ in range(max(3, args.warmup)):
+            call()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b) / 1e3)
+        if sdpa.get_last_device_error() != sdpa.SDPA_OK:
+            raise SystemExit("device error in backward")
+        t = float(np.mean(times))
+        flops = 2.5 * w.flops()
+        peak = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+        res[w.name] = {"value": round(flops / t / 1e12, 1), "unit": "TFLOP/s", "ms": round(t * 1e3, 4),
+                       "gpu_launches_per_call": 3,
+                       "roofline": {"kernel": "sdpa_bwd_pre + sdpa_bwd_dkdv + sdpa_bwd_dq", "bound": "tensor",
+                                    "achieved": round(flops / t / 1e12, 1), "peak": peak, "unit": "TFLOP/s",
+                                    "frac": round(flops / t / 1e12 / peak, 4),
+                                    "peak_kind": peak_kind + " burst bf16", "algorithmic_flop": flops,
+                                    "executed_flop": 3.5 * w.flops(), "traffic": None}}
+    del dq, dk, dv, ws, do
+    return res
+
+
+def run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, grouped=False):
+    """Decode sub-benchmark: cfg5 (one key/value head per query head) or, grouped, cfg5g."""
+    import torch
+    w = W.CFG5G if grouped else W.CFG5
     if args.decode_batch != w.batch:  # same recipe, fewer sequences (e.g. to keep a profiler capture small)
-        w = W.Decode("cfg5_b%d" % args.decode_batch, args.decode_batch, w.heads, w.n_cap, w.d, w.len_lo, w.len_hi,
-                     w.scale, w.seed)
+        w = W.Decode("%s_b%d" % (w.name, args.decode_batch), args.decode_batch, w.heads, w.n_cap, w.d, w.len_lo,
+                     w.len_hi, w.scale, w.seed, w.heads_kv)
     lens = w.lengths()
     tl = torch.from_numpy(lens).to(dev)
-    shape = (w.batch, w.heads, w.n_cap, w.d)
+    shape = (w.batch, w.kv_heads, w.n_cap, w.d)
     kc = torch.empty(shape, dtype=torch.bfloat16, device=dev)
     vc = torch.empty(shape, dtype=torch.bfloat16, device=dev)
     si.fill_device_cache(kc, tl, w.seed, si.STREAM_K)
@@ -366,8 +448,13 @@ def run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind):
     q = W.to_torch(si.fill_host((w.batch, w.heads, w.d), w.seed, si.STREAM_Q), dev)
     o = torch.empty_like(q)
     lse = torch.empty((w.batch, w.heads), dtype=torch.float32, device=dev)
-    ws = torch.empty(sdpa.decode_workspace_size(w.batch, w.heads, w.n_cap, w.d), dtype=torch.uint8, device=dev)
-    call = lambda: sdpa.decode(q, kc, vc, tl, scale=w.scale_f32, o=o, lse=lse, workspace=ws, stream=stream)
+    if grouped:
+        ws = torch.empty(sdpa.decode_gqa_workspace_size(w.batch, w.heads, w.kv_heads, w.n_cap, w.d),
+                         dtype=torch.uint8, device=dev)
+        call = lambda: sdpa.decode_gqa(q, kc, vc, tl, scale=w.scale_f32, o=o, lse=lse, workspace=ws, stream=stream)
+    else:
+        ws = torch.empty(sdpa.decode_workspace_size(w.batch, w.heads, w.n_cap, w.d), dtype=torch.uint8, device=dev)
+        call = lambda: sdpa.decode(q, kc, vc, tl, scale=w.scale_f32, o=o, lse=lse, workspace=ws, stream=stream)
     for _ in range(max(3, args.warmup)):
         call()
     torch.cuda.synchronize()
@@ -387,13 +474,20 @@ def run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind):
     peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
     del kc, vc
     torch.cuda.empty_cache()
-    return {"workload": "%s: decode bf16 batch %d x 32 heads, cache 16384, lengths U{1024..16384} "
-                        "(sum %d), d = 128" % (w.name, w.batch, int(lens.sum())),
+    heads = ("%d query heads over %d key/value heads" % (w.heads, w.kv_heads)) if grouped else "%d heads" % w.heads
+    if grouped:
+        kernel, prof, srcs = "sdpa_decode_gqa_kernel<16> + combine", "decode_cfg5g_dram.txt", GQA_SOURCES
+    else:
+        kernel, prof, srcs = "sdpa_decode_split_kernel + combine", "decode_cfg5_dram.txt", DECODE_SOURCES
+    return {"workload": "%s: decode bf16 batch %d x %s, cache 16384, lengths U{1024..16384} (sum %d), d = 128"
+                        % (w.name, w.batch, heads, int(lens.sum())),
             "value": round(gbs, 1), "unit": "GB/s", "ms": round(t * 1e3, 4), "gpu_launches_per_call": 2,
-            "roofline": {"kernel": "sdpa_decode_split_kernel + combine", "bound": "hbm", "achieved": round(gbs, 1),
+            "gflops": round(w.flops(lens) / t / 1e9, 1),
+            "cost_model": cost_model(w.flops(lens), w.bytes(lens), t, peaks),
+            "roofline": {"kernel": kernel, "bound": "hbm", "achieved": round(gbs, 1),
                          "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
                          "peak_kind": peak_kind + " HBM copy",
-                         "traffic": (None if w.batch != 64 else profiled_traffic("decode_cfg5_dram.txt", DECODE_SOURCES)),
+                         "traffic": (None if args.decode_batch != 64 else profiled_traffic(prof, srcs)),
                          "algorithmic_bytes": w.bytes(lens)}}
 
 
@@ -438,6 +532,7 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=64, help="sequences in the decode workload (default 64)")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -165,6 +165,56 @@ SDPA_API int sdpa_decode_noalloc(const void* Q, const void* K, const void* V, co
                                  void* stream);
 
 /*
+ * sdpa_bwd_workspace_size -- bytes of device workspace sdpa_bwd needs:
+ * 2 * batch * heads * round_up(n_q, 128) floats.  0 for a degenerate shape.
+ */
+SDPA_API size_t sdpa_bwd_workspace_size(int batch, int heads, int n_q);
+
+/*
+ * sdpa_bwd -- gradients of sdpa_fwd: dQ, dK, dV for the loss gradient dO, from the forward's
+ * inputs, its output O and its LSE (the MoA roadmap's last stage, a backward pass in the same
+ * memory-optimal form: agents-report.net MoA article, "implementation roadmap").
+ *
+ * With P = softmax(Q K^T scale) recomputed from LSE, D_i = dO_i . O_i and dS = P (dO V^T - D):
+ *   dV = P^T dO,   dK = scale dS^T Q,   dQ = scale dS K.
+ * Nothing of size n_q x n_kv is written; each gradient is written once.
+ * Q, O, dO, dQ [batch, heads, n_q, d]; K, V, dK, dV [batch, heads, n_kv, d]; all
+ * __nv_bfloat16, contiguous, 16-byte aligned.  LSE [batch, heads, n_q] float as sdpa_fwd wrote
+ * it (required).  d_k == d_v in {64, 128}; scale > 0 and causal as in the forward call.
+ * workspace: caller-owned device memory of sdpa_bwd_workspace_size bytes (scratch).
+ * Rows whose window held no key (causal, n_q > n_kv) contribute nothing and get dQ = 0.
+ * Errors as sdpa_fwd, plus SDPA_ERR_WORKSPACE.
+ */
+SDPA_API int sdpa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                      void* dQ, void* dK, void* dV, int batch, int heads, int n_q, int n_kv, int d_k, int d_v,
+                      float scale, int causal, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * sdpa_decode_gqa_workspace_size -- bytes of device workspace sdpa_decode_gqa needs for
+ * this shape; 0 for a degenerate or invalid one (heads_q not a multiple of heads_kv).
+ */
+SDPA_API size_t sdpa_decode_gqa_workspace_size(int batch, int heads_q, int heads_kv, int n_kv_cap, int d_v);
+
+/*
+ * sdpa_decode_gqa -- grouped-query decode: heads_q query heads share heads_kv key/value
+ * heads, query head h reading key/value head h / (heads_q / heads_kv) (consecutive query
+ * heads form a group).  Grouped-query layouts are what let the 2-simplicial article
+ * (szyisi.cn, "model design") tile along query heads into dense products; here each
+ * group's keys and values are read from HBM once for all of its query heads.
+ *
+ * Q [batch, heads_q, d_k]; K [batch, heads_kv, n_kv_cap, d_k]; V [batch, heads_kv,
+ * n_kv_cap, d_v]; O [batch, heads_q, d_v], all __nv_bfloat16; LSE [batch, heads_q] float
+ * or NULL.  kv_lens, alignment, workspace ownership and errors as sdpa_decode, with the
+ * workspace sized by sdpa_decode_gqa_workspace_size.  heads_q % heads_kv != 0 is
+ * SDPA_ERR_INVALID_ARG.  d_k == d_v == 128 with 2 to 32 query heads per group runs on
+ * the tensor cores (tcgen05); other groups and d = 64 run the CUDA-core split kernel
+ * with the same head mapping.  heads_q == heads_kv is sdpa_decode.
+ */
+SDPA_API int sdpa_decode_gqa(const void* Q, const void* K, const void* V, const int* kv_lens, void* O, float* LSE,
+                             int batch, int heads_q, int heads_kv, int n_kv_cap, int d_k, int d_v, float scale,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * sdpa_get_last_device_error -- synchronise `stream`, then read and clear the
  * device error word of the current device.  Returns SDPA_OK, the first device
  * error recorded since the last call, or SDPA_ERR_CUDA if the synchronisation

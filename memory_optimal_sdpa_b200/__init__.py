@@ -8,6 +8,8 @@ fallback: if libsdpa.so is missing, importing this package fails.
     O, LSE = sdpa.fwd(q, k, v, causal=True)                 # bf16, tcgen05 tensor cores
     O, LSE = sdpa.fwd_f32(q, k, v)                          # fp32 on CUDA cores
     O, LSE = sdpa.decode(q, k_cache, v_cache, kv_lens)      # one row per (batch, head)
+    O, LSE = sdpa.decode_gqa(q, k_cache, v_cache, kv_lens)  # query heads sharing key/value heads
+    dQ, dK, dV = sdpa.bwd(q, k, v, O, dO, LSE, causal=True) # gradients of fwd
 """
 import ctypes
 import math
@@ -35,6 +37,14 @@ lib.sdpa_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f
 lib.sdpa_decode.restype = _i
 lib.sdpa_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp]
 lib.sdpa_decode_noalloc.restype = _i
+lib.sdpa_decode_gqa_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+lib.sdpa_decode_gqa_workspace_size.restype = _sz
+lib.sdpa_decode_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]
+lib.sdpa_decode_gqa.restype = _i
+lib.sdpa_bwd_workspace_size.argtypes = [_i, _i, _i]
+lib.sdpa_bwd_workspace_size.restype = _sz
+lib.sdpa_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _vp, _sz, _vp]
+lib.sdpa_bwd.restype = _i
 lib.sdpa_get_last_device_error.argtypes = [_vp]
 lib.sdpa_get_last_device_error.restype = _i
 lib.sdpa_status_string.argtypes = [_i]
@@ -159,6 +169,54 @@ def decode_noalloc(q, k, v, kv_lens, scale=None, o=None, lse=None, want_lse=True
     _check(lib.sdpa_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), _ptr(o), _ptr(lse), B, H, n_cap, d_k,
                                    d_v, float(scale), _stream(stream)), "sdpa_decode_noalloc")
     return o, lse
+
+
+def decode_gqa_workspace_size(batch, heads_q, heads_kv, n_kv_cap, d_v):
+    return int(lib.sdpa_decode_gqa_workspace_size(batch, heads_q, heads_kv, n_kv_cap, d_v))
+
+
+def decode_gqa(q, k, v, kv_lens, scale=None, o=None, lse=None, want_lse=True, workspace=None, stream=None):
+    """Grouped-query decode. q [B, H_q, d], k/v [B, H_kv, n_cap, d] bf16 (H_q a multiple of H_kv),
+    kv_lens int32 [B] on the device; query head h reads key/value head h // (H_q // H_kv)."""
+    import torch
+    B, H_kv, n_cap, d_k = k.shape
+    H_q = q.shape[1]
+    d_v = v.shape[3]
+    scale = 1.0 / math.sqrt(d_k) if scale is None else scale
+    if o is None:
+        o = torch.empty((B, H_q, d_v), dtype=q.dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=q.device)
+    need = decode_gqa_workspace_size(B, H_q, H_kv, n_cap, d_v)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib.sdpa_decode_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), _ptr(o), _ptr(lse), B, H_q, H_kv, n_cap,
+                               d_k, d_v, float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream)), "sdpa_decode_gqa")
+    return o, lse
+
+
+def bwd_workspace_size(batch, heads, n_q):
+    return int(lib.sdpa_bwd_workspace_size(batch, heads, n_q))
+
+
+def bwd(q, k, v, o, do, lse, causal=False, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of fwd: returns dQ, dK, dV (bf16, shapes of q, k, v) for loss gradient `do`,
+    from the forward's inputs, output `o` and `lse`."""
+    import torch
+    B, H, n_q, d_k = q.shape
+    n_kv, d_v = v.shape[2], v.shape[3]
+    scale = 1.0 / math.sqrt(d_k) if scale is None else scale
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_size(B, H, n_q)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib.sdpa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, H,
+                        n_q, n_kv, d_k, d_v, float(scale), int(bool(causal)), _ptr(workspace),
+                        workspace.numel() * workspace.element_size(), _stream(stream)), "sdpa_bwd")
+    return dq, dk, dv
 
 
 def get_last_device_error(stream=None):

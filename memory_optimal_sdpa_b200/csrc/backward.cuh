@@ -1,0 +1,589 @@
+// backward.cuh -- gradients of exact SDPA (dQ, dK, dV), bf16 in and out, on the sm_100a tensor cores.
+//
+// The MoA roadmap ends with the backward pass in the same memory-optimal form
+// (agents-report.net MoA article, "implementation roadmap").  Given the saved
+// log-sum-exp of every query row, the probabilities are recomputed tile by tile
+// and nothing of size n_q x n_kv reaches memory:
+//   P  = exp(S scale - LSE)            S = Q K^T
+//   dP = dO V^T,   D_i = dO_i . O_i    (= sum_k P_ik dP_ik)
+//   dS = P (dP - D)
+//   dV = P^T dO,   dK = scale dS^T Q,   dQ = scale dS K
+// Three kernels:
+//   pre   D_i and LSE in log2 units (+inf where a row must get P = 0) into a workspace
+//   dkdv  one CTA per 128-key tile, streaming the query tiles that see it:
+//         S^T = K Q^T and dP^T = V dO^T (tcgen05, fp32 in TMEM), the elementwise
+//         P^T and dS^T (bf16, written back over S^T and dP^T), then dV += P^T dO and
+//         dK += dS^T Q with the TMEM operand form; dV and dK stay in TMEM to the end
+//   dq    one CTA per 128-row query tile, streaming key tiles: S, dP, dS as above,
+//         then dQ += dS K
+// Each gradient is written once, so global traffic is O(n d) per kernel and no
+// atomics are needed; the price is computing S and dP in both kernels.
+//
+// Warp roles (384 threads, as the forward kernel): warps 0-7 two elementwise
+// warpgroups (warpgroup w takes columns [64 w, 64 w + 64) of the 128 x 128
+// tile; thread = TMEM lane = the tile's key (dkdv) or query row (dq)), warp 8
+// the TMA producer, warp 9 the MMA issuer and TMEM owner, warps 10-11 idle.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+
+namespace sdpa {
+
+struct BwdParams {
+  const __nv_bfloat16* O;   // [bh, n_q, D]   (pre)
+  const __nv_bfloat16* dO;  // [bh, n_q, D]   (pre)
+  const float* LSE;         // [bh, n_q], natural log of the scaled logits (pre)
+  float* Dvec;              // [bh, n_q_pad]  rowsum(dO * O); 0 in the padding
+  float* L2;                // [bh, n_q_pad]  LSE * log2(e); +inf in the padding and for rows without keys
+  __nv_bfloat16* dQ;        // [bh, n_q, D]
+  __nv_bfloat16* dK;        // [bh, n_kv, D]
+  __nv_bfloat16* dV;        // [bh, n_kv, D]
+  int n_q, n_kv, n_q_pad, bh_count;
+  float scale, scale_log2;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int BLOCK_BYTES = 128 * 64 * 2;
+  // d = 64: four stages, which also keeps the CTA's shared memory above half an SM's, so a
+  // second CTA (that would wait for TMEM) is never placed beside it.
+  static constexpr int NSTAGE = (D == 64) ? 4 : 2;
+  static constexpr int VEC_BYTES = 1024;  // L2[128] then D[128] of a query tile (dkdv only)
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES + VEC_BYTES;
+  static constexpr int FIX_OFF = 0;                // the CTA's fixed pair: (K, V) or (Q, dO)
+  static constexpr int ST_OFF = 2 * TILE_BYTES;    // streamed stages: (Q, dO, vectors) or (K, V)
+  static constexpr int BAR_OFF = ST_OFF + NSTAGE * STAGE_BYTES;
+  // fix_full, full[NSTAGE], empty[NSTAGE], s_full, p_full[2], o_full, drain
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 5;
+  static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;
+  static constexpr int THREADS = 384;
+  static constexpr int EW_REGS = 216;
+  static constexpr int CONTROL_REGS = 72;
+  static constexpr int LOAD_WARP = 8;
+  static constexpr int MMA_WARP = 9;
+  static constexpr uint32_t COL_S = 0;      // S or S^T, fp32; then P^T (bf16 pairs) over its first columns
+  static constexpr uint32_t COL_DP = 128;   // dP or dP^T, fp32; then dS / dS^T (bf16 pairs)
+  static constexpr uint32_t COL_A = 256;    // accumulator: dV (dkdv) or dQ (dq)
+  static constexpr uint32_t COL_B = 256 + D;  // accumulator: dK (dkdv)
+  static constexpr uint32_t TMEM_COLS = 512;
+};
+
+// TMEM column of the bf16 pairs holding tile columns [16 kk, 16 kk + 16): warpgroup w packs
+// its 64 columns into [64 w, 64 w + 32) of the fp32 region it read them from.
+__device__ __forceinline__ uint32_t bwd_pair_col(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
+
+// ------------------------------------------------------------------------------------ pre
+template <int D>
+__global__ void __launch_bounds__(128) sdpa_bwd_pre_kernel(const BwdParams p) {
+  constexpr int LPR = D / 8;      // lanes per row, 8 elements each
+  constexpr int RPW = 32 / LPR;   // rows per warp pass
+  const int bh = blockIdx.y;
+  const int r0 = blockIdx.x * 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e0 = (lane % LPR) * 8;
+  const float POS_INF = __int_as_float(0x7f800000);
+  for (int it = 0; it < 128 / (4 * RPW); ++it) {
+    const int row = r0 + (it * 4 + warp) * RPW + lane / LPR;
+    float dot = 0.f;
+    if (row < p.n_q) {
+      const size_t off = ((size_t)bh * p.n_q + row) * D + e0;
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(p.O + off));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.dO + off));
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        dot = fmaf(__uint_as_float(wa[i] << 16), __uint_as_float(wb[i] << 16), dot);
+        dot = fmaf(__uint_as_float(wa[i] & 0xFFFF0000u), __uint_as_float(wb[i] & 0xFFFF0000u), dot);
+      }
+    }
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (lane % LPR == 0) {
+      const size_t o = (size_t)bh * p.n_q_pad + row;
+      if (row < p.n_q) {
+        const float lse = p.LSE[(size_t)bh * p.n_q + row];
+        p.Dvec[o] = dot;
+        p.L2[o] = (lse == -POS_INF) ? POS_INF : lse * 1.4426950408889634f;  // no key: P = 0 everywhere
+      } else {
+        p.Dvec[o] = 0.f;
+        p.L2[o] = POS_INF;
+      }
+    }
+  }
+}
+
+// Elementwise step shared by both kernels, for 32 tile columns starting at `c0` of this
+// warpgroup's half: P = 2^(S c2 - l2), dS = P (dP - dd), with `keep(c)` false for masked
+// entries.  s and dp hold the 32 fp32 values; pp and ps receive the bf16 pairs.
+template <class L2F, class DDF, class KEEP>
+__device__ __forceinline__ void bwd_elementwise(const uint32_t (&s)[32], const uint32_t (&dp)[32], float c2,
+                                                L2F l2, DDF dd, KEEP keep, uint32_t (&pp)[16],
+                                                uint32_t (&ps)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float pr[2], dr[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = 2 * i + h;
+      float e = sm100::ex2_approx(__uint_as_float(s[c]) * c2 - l2(c));
+      if (!keep(c)) e = 0.f;
+      pr[h] = e;
+      dr[h] = e * (__uint_as_float(dp[c]) - dd(c));
+    }
+    pp[i] = sm100::pack_bf16x2(pr[0], pr[1]);
+    ps[i] = sm100::pack_bf16x2(dr[0], dr[1]);
+  }
+}
+
+// ------------------------------------------------------------------------------------ dK, dV
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    sdpa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                         const BwdParams p) {
+  using C = BwdCfg<D>;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sFix = smem + C::FIX_OFF;  // K, V
+  uint8_t* sSt = smem + C::ST_OFF;    // per stage: Q, dO, L2[128], D[128]
+  uint64_t* bars = (uint64_t*)(smem + C::BAR_OFF);
+  uint64_t* fix_full = bars;
+  uint64_t* full = bars + 1;
+  uint64_t* empty = full + C::NSTAGE;
+  uint64_t* s_full = empty + C::NSTAGE;
+  uint64_t* p_full = s_full + 1;  // [warpgroup]
+  uint64_t* o_full = p_full + 2;
+  uint64_t* drain = o_full + 1;
+  uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x % p.bh_count;
+  const int j0 = (int)(blockIdx.x / p.bh_count) * 128;  // key tile (causal: the first ones see the most rows)
+  const int off = p.n_kv - p.n_q;                        // bottom-right alignment
+  // Query tiles that see some key of [j0, j0 + 128): causal rows q with q + off >= j0.
+  int t_first = 0;
+  if (CAUSAL) {
+    const long long q_min = (long long)j0 - off;
+    t_first = q_min <= 0 ? 0 : (int)(q_min / 128);
+  }
+  const int n_qt = (p.n_q + 127) / 128;
+  const int NT = t_first < n_qt ? n_qt - t_first : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(fix_full, 1);
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(&p_full[0], 128);
+    mbar_init(&p_full[1], 128);
+    mbar_init(o_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool timed_out = false;
+  static_assert(C::EW_REGS * 256 + C::CONTROL_REGS * 128 <= 168 * 384, "register split exceeds the launch");
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONTROL_REGS));
+    if (warp == C::LOAD_WARP) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0 && NT > 0) {
+        mbar_arrive_expect_tx(fix_full, 2 * C::TILE_BYTES);
+#pragma unroll
+        for (int cb = 0; cb < D / 64; ++cb) {
+          tma_load_3d(sFix + cb * C::BLOCK_BYTES, &tmK, fix_full, cb * 64, j0, bh);
+          tma_load_3d(sFix + C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmV, fix_full, cb * 64, j0, bh);
+        }
+        int issued = 0;
+        for (int t = 0; t < NT; ++t) {
+          const int st = t % C::NSTAGE;
+          if (!mbar_wait_bounded(&empty[st], ((uint32_t)(t / C::NSTAGE) & 1u) ^ 1u, abort_flag, &timed_out)) break;
+          uint8_t* dst = sSt + st * C::STAGE_BYTES;
+          const int q0 = (t_first + t) * 128;
+          mbar_arrive_expect_tx(&full[st], 2 * C::TILE_BYTES + C::VEC_BYTES);
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb) {
+            tma_load_3d(dst + cb * C::BLOCK_BYTES, &tmQ, &full[st], cb * 64, q0, bh);
+            tma_load_3d(dst + C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmdO, &full[st], cb * 64, q0, bh);
+          }
+          const size_t v0 = (size_t)bh * p.n_q_pad + q0;
+          bulk_load(dst + 2 * C::TILE_BYTES, p.L2 + v0, 512, &full[st]);
+          bulk_load(dst + 2 * C::TILE_BYTES + 512, p.Dvec + v0, 512, &full[st]);
+          issued = t + 1;
+        }
+        if (*abort_flag) {  // let the copies in flight land before the CTA exits
+          mbar_wait_drain(fix_full, 0);
+          for (int t = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); t < issued; ++t)
+            mbar_wait_drain(&full[t % C::NSTAGE], (uint32_t)(t / C::NSTAGE) & 1u);
+        }
+      }
+    } else if (warp == C::MMA_WARP) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0 && NT > 0) {
+        constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // K or V (K-major) x Q or dO (K-major)
+        constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);     // P^T or dS^T (TMEM) x dO or Q (MN-major)
+        const uint32_t fix = smem_u32(sFix), st0 = smem_u32(sSt);
+        const uint64_t dK = smem_desc_sw128(fix, 16, 1024);
+        const uint64_t dV = smem_desc_sw128(fix + C::TILE_BYTES, 16, 1024);
+        auto wait_bar = [&](uint64_t* bar, int phase) {
+          return mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
+        };
+        bool ok = wait_bar(fix_full, 0);
+        for (int t = 0; ok && t < NT; ++t) {
+          const int st = t % C::NSTAGE;
+          const uint32_t sq = st0 + st * C::STAGE_BYTES, sdo = sq + C::TILE_BYTES;
+          if (!(ok = wait_bar(&full[st], t / C::NSTAGE))) break;
+          const uint64_t dQk = smem_desc_sw128(sq, 16, 1024), dOk = smem_desc_sw128(sdo, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K Q^T, dP^T = V dO^T
+            const uint64_t o = (uint64_t)((((kk >> 2) * C::BLOCK_BYTES) + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + C::COL_S, dK + o, dQk + o, idS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_DP, dV + o, dOk + o, idS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full);
+          const uint64_t dOm = smem_desc_sw128(sdo, C::BLOCK_BYTES, 1024);  // MN-major views
+          const uint64_t dQm = smem_desc_sw128(sq, C::BLOCK_BYTES, 1024);
+          for (int w = 0; ok && w < 2; ++w) {  // each warpgroup's 64 query columns as soon as they are ready
+            if (!(ok = wait_bar(&p_full[w], t))) break;
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int kk = 4 * w + k4;
+              const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+              const uint64_t ob = (uint64_t)((kk * 2048) >> 4);
+              mma_ts(tmem + C::COL_A, tmem + C::COL_S + bwd_pair_col(kk), dOm + ob, idA, acc);   // dV += P^T dO
+              mma_ts(tmem + C::COL_B, tmem + C::COL_DP + bwd_pair_col(kk), dQm + ob, idA, acc);  // dK += dS^T Q
+            }
+          }
+          if (!ok) break;
+          tc_commit(&empty[st]);
+        }
+        if (ok) tc_commit(o_full);
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0);
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::EW_REGS));
+    // ------------------------------------------------------- elementwise + epilogue
+    const int w = warp >> 2;           // column half of the tile
+    const int row = 32 * (warp & 3) + lane;  // TMEM lane = key within the tile
+    const int key = j0 + row;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const float c2 = p.scale_log2;
+    bool ok = true;
+    auto wait_warp = [&](uint64_t* bar, int phase) {
+      const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
+      return __all_sync(0xffffffffu, r);
+    };
+    for (int t = 0; ok && t < NT; ++t) {
+      const int st = t % C::NSTAGE;
+      const float* vL2 = reinterpret_cast<const float*>(sSt + st * C::STAGE_BYTES + 2 * C::TILE_BYTES);
+      const float* vD = vL2 + 128;
+      // the stage's vectors come from the bulk copy: wait for it here too, not only through the MMAs
+      if (!(ok = wait_warp(&full[st], t / C::NSTAGE) && wait_warp(s_full, t))) break;
+      tc_fence_after_sync();
+      const int q0 = (t_first + t) * 128 + 64 * w;  // first query of this warpgroup's columns
+      const bool masked = CAUSAL && (q0 + off < j0 + 127);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int cbase = 64 * w + 32 * h;  // tile column of this chunk
+        uint32_t s[32], dp[32];
+        tmem_ld_32x32b_x32(tmem + C::COL_S + (uint32_t)cbase + lane_base, s);
+        tmem_ld_32x32b_x32(tmem + C::COL_DP + (uint32_t)cbase + lane_base, dp);
+        tmem_wait_ld();
+        reg_fence(s);
+        reg_fence(dp);
+        uint32_t pp[16], ps[16];
+        const int qc = q0 + 32 * h;
+        if (masked)
+          bwd_elementwise(s, dp, c2, [&](int c) { return vL2[cbase + c]; }, [&](int c) { return vD[cbase + c]; },
+                          [&](int c) { return key <= qc + c + off; }, pp, ps);
+        else
+          bwd_elementwise(s, dp, c2, [&](int c) { return vL2[cbase + c]; }, [&](int c) { return vD[cbase + c]; },
+                          [&](int) { return true; }, pp, ps);
+        tmem_st_32x32b_x16(tmem + C::COL_S + (uint32_t)(64 * w + 16 * h) + lane_base, pp);
+        tmem_st_32x32b_x16(tmem + C::COL_DP + (uint32_t)(64 * w + 16 * h) + lane_base, ps);
+      }
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(&p_full[w]);
+    }
+    // ---------------------------------------------------------------- epilogue
+    if (ok && NT > 0) ok = wait_warp(o_full, 0);
+    if (ok) {
+      tc_fence_after_sync();
+      // warpgroup 0 writes dV, warpgroup 1 writes dK (times scale); zeros if no query sees the tile
+      const uint32_t col = w ? C::COL_B : C::COL_A;
+      const float mul = w ? p.scale : 1.f;
+      const bool store = key < p.n_kv;
+      __nv_bfloat16* dst = (w ? p.dK : p.dV) + ((size_t)bh * p.n_kv + (store ? key : 0)) * D;
+#pragma unroll 1
+      for (int cb = 0; cb < D; cb += 32) {
+        uint32_t o[32];
+        if (NT > 0) {
+          tmem_ld_32x32b_x32(tmem + col + (uint32_t)cb + lane_base, o);
+          tmem_wait_ld();
+          reg_fence(o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        uint32_t v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          v[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * mul, __uint_as_float(o[2 * i + 1]) * mul);
+        if (store) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + cb);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+    }
+  }
+
+  if (timed_out) record_error(6 /* SDPA_ERR_DEVICE_TIMEOUT */);
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------ dQ
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    sdpa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                       const BwdParams p) {
+  using C = BwdCfg<D>;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sFix = smem + C::FIX_OFF;  // Q, dO
+  uint8_t* sSt = smem + C::ST_OFF;    // per stage: K, V
+  uint64_t* bars = (uint64_t*)(smem + C::BAR_OFF);
+  uint64_t* fix_full = bars;
+  uint64_t* full = bars + 1;
+  uint64_t* empty = full + C::NSTAGE;
+  uint64_t* s_full = empty + C::NSTAGE;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* drain = o_full + 1;
+  uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x % p.bh_count;
+  const int n_qt = (p.n_q + 127) / 128;
+  const int q0 = (n_qt - 1 - (int)(blockIdx.x / p.bh_count)) * 128;  // causal: the last rows see the most keys
+  const int off = p.n_kv - p.n_q;
+  int T = (p.n_kv + 127) / 128;  // key tiles this query tile visits
+  if (CAUSAL) {
+    const int last_row = (q0 + 127 < p.n_q - 1) ? q0 + 127 : p.n_q - 1;
+    const long long max_key = (long long)last_row + off;
+    T = max_key < 0 ? 0 : (int)(max_key / 128) + 1 < T ? (int)(max_key / 128) + 1 : T;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(fix_full, 1);
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(&p_full[0], 128);
+    mbar_init(&p_full[1], 128);
+    mbar_init(o_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool timed_out = false;
+  static_assert(C::EW_REGS * 256 + C::CONTROL_REGS * 128 <= 168 * 384, "register split exceeds the launch");
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONTROL_REGS));
+    if (warp == C::LOAD_WARP) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0 && T > 0) {
+        mbar_arrive_expect_tx(fix_full, 2 * C::TILE_BYTES);
+#pragma unroll
+        for (int cb = 0; cb < D / 64; ++cb) {
+          tma_load_3d(sFix + cb * C::BLOCK_BYTES, &tmQ, fix_full, cb * 64, q0, bh);
+          tma_load_3d(sFix + C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmdO, fix_full, cb * 64, q0, bh);
+        }
+        int issued = 0;
+        for (int j = 0; j < T; ++j) {
+          const int st = j % C::NSTAGE;
+          if (!mbar_wait_bounded(&empty[st], ((uint32_t)(j / C::NSTAGE) & 1u) ^ 1u, abort_flag, &timed_out)) break;
+          uint8_t* dst = sSt + st * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[st], 2 * C::TILE_BYTES);
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb) {
+            tma_load_3d(dst + cb * C::BLOCK_BYTES, &tmK, &full[st], cb * 64, j * 128, bh);
+            tma_load_3d(dst + C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmV, &full[st], cb * 64, j * 128, bh);
+          }
+          issued = j + 1;
+        }
+        if (*abort_flag) {
+          mbar_wait_drain(fix_full, 0);
+          for (int j = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); j < issued; ++j)
+            mbar_wait_drain(&full[j % C::NSTAGE], (uint32_t)(j / C::NSTAGE) & 1u);
+        }
+      }
+    } else if (warp == C::MMA_WARP) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0 && T > 0) {
+        constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q or dO (K-major) x K or V (K-major)
+        constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);     // dS (TMEM) x K (MN-major)
+        const uint32_t fix = smem_u32(sFix), st0 = smem_u32(sSt);
+        const uint64_t dQk = smem_desc_sw128(fix, 16, 1024);
+        const uint64_t dOk = smem_desc_sw128(fix + C::TILE_BYTES, 16, 1024);
+        auto wait_bar = [&](uint64_t* bar, int phase) {
+          return mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
+        };
+        bool ok = wait_bar(fix_full, 0);
+        for (int j = 0; ok && j < T; ++j) {
+          const int st = j % C::NSTAGE;
+          const uint32_t sk = st0 + st * C::STAGE_BYTES, sv = sk + C::TILE_BYTES;
+          if (!(ok = wait_bar(&full[st], j / C::NSTAGE))) break;
+          const uint64_t dKk = smem_desc_sw128(sk, 16, 1024), dVk = smem_desc_sw128(sv, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {  // S = Q K^T, dP = dO V^T
+            const uint64_t o = (uint64_t)((((kk >> 2) * C::BLOCK_BYTES) + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + C::COL_S, dQk + o, dKk + o, idS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_DP, dOk + o, dVk + o, idS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full);
+          const uint64_t dKm = smem_desc_sw128(sk, C::BLOCK_BYTES, 1024);
+          for (int w = 0; ok && w < 2; ++w) {
+            if (!(ok = wait_bar(&p_full[w], j))) break;
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int kk = 4 * w + k4;
+              mma_ts(tmem + C::COL_A, tmem + C::COL_DP + bwd_pair_col(kk), dKm + (uint64_t)((kk * 2048) >> 4), idA,
+                     (j > 0 || kk > 0) ? 1u : 0u);  // dQ += dS K
+            }
+          }
+          if (!ok) break;
+          tc_commit(&empty[st]);
+        }
+        if (ok) tc_commit(o_full);
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0);
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::EW_REGS));
+    // ------------------------------------------------------- elementwise + epilogue
+    const int w = warp >> 2;                 // column half: keys [64 w, 64 w + 64) of each tile
+    const int row = 32 * (warp & 3) + lane;  // TMEM lane = query row within the tile
+    const int q = q0 + row;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const float c2 = p.scale_log2;
+    const size_t vi = (size_t)bh * p.n_q_pad + q;  // inside the padded vectors for every lane
+    const float l2 = p.L2[vi];
+    const float dd = p.Dvec[vi];
+    bool ok = true;
+    auto wait_warp = [&](uint64_t* bar, int phase) {
+      const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
+      return __all_sync(0xffffffffu, r);
+    };
+    for (int j = 0; ok && j < T; ++j) {
+      if (!(ok = wait_warp(s_full, j))) break;
+      tc_fence_after_sync();
+      const int k0 = j * 128 + 64 * w;  // first key of this warpgroup's columns
+      const bool masked = (k0 + 63 >= p.n_kv) || (CAUSAL && k0 + 63 > q0 + off);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int cbase = 64 * w + 32 * h;
+        uint32_t s[32], dp[32];
+        tmem_ld_32x32b_x32(tmem + C::COL_S + (uint32_t)cbase + lane_base, s);
+        tmem_ld_32x32b_x32(tmem + C::COL_DP + (uint32_t)cbase + lane_base, dp);
+        tmem_wait_ld();
+        reg_fence(s);
+        reg_fence(dp);
+        uint32_t pp[16], ps[16];
+        const int kc = k0 + 32 * h;
+        if (masked)
+          bwd_elementwise(s, dp, c2, [&](int) { return l2; }, [&](int) { return dd; },
+                          [&](int c) { return kc + c < p.n_kv && (!CAUSAL || kc + c <= q + off); }, pp, ps);
+        else
+          bwd_elementwise(s, dp, c2, [&](int) { return l2; }, [&](int) { return dd; }, [&](int) { return true; }, pp,
+                          ps);
+        tmem_st_32x32b_x16(tmem + C::COL_DP + (uint32_t)(64 * w + 16 * h) + lane_base, ps);
+      }
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(&p_full[w]);
+    }
+    // ---------------------------------------------------------------- epilogue
+    if (ok && T > 0) ok = wait_warp(o_full, 0);
+    if (ok) {
+      tc_fence_after_sync();
+      // warpgroup w writes columns [w D/2, w D/2 + D/2) of this row's dQ (times scale)
+      const bool store = q < p.n_q;
+      __nv_bfloat16* dst = p.dQ + ((size_t)bh * p.n_q + (store ? q : 0)) * D;
+#pragma unroll 1
+      for (int cb = w * (D / 2); cb < (w + 1) * (D / 2); cb += 32) {
+        uint32_t o[32];
+        if (T > 0) {
+          tmem_ld_32x32b_x32(tmem + C::COL_A + (uint32_t)cb + lane_base, o);
+          tmem_wait_ld();
+          reg_fence(o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        uint32_t v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          v[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * p.scale, __uint_as_float(o[2 * i + 1]) * p.scale);
+        if (store) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + cb);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+    }
+  }
+
+  if (timed_out) record_error(6 /* SDPA_ERR_DEVICE_TIMEOUT */);
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace sdpa

@@ -6,6 +6,10 @@
 // self-attention"): a bandwidth-bound stream, so the kernel is built around
 // HBM reads, not arithmetic.
 //
+// Grouped-query attention (query head h reading key/value head h / group) uses the
+// same kernel with a group size above one; the tensor-core kernel in
+// decode_gqa.cuh takes the common d = 128 groups.
+//
 // Split-KV: CTA (split s, head h, batch b) reduces keys [s*chunk, (s+1)*chunk)
 // of row b's valid prefix [0, len_b) to a partial (O_s normalised, lse_s).
 // Each key is handled by D/8 lanes holding 8 dimensions each (one 16-byte
@@ -59,7 +63,7 @@ __device__ __forceinline__ int decode_len(const int* kv_lens, int b, int n_cap) 
 
 struct DecodeParams {
   const __nv_bfloat16* Q;  // [B, H, D]
-  const __nv_bfloat16* K;  // [B, H, n_cap, D]
+  const __nv_bfloat16* K;  // [B, H_kv, n_cap, D]: query head h reads key/value head h / group
   const __nv_bfloat16* V;
   const int* kv_lens;      // [B]
   float* part_o;           // [B, H, S, D]
@@ -67,6 +71,7 @@ struct DecodeParams {
   __nv_bfloat16* O;        // [B, H, D]
   float* LSE;              // [B, H] or null
   int H, n_cap, chunk, n_split;
+  int H_kv, group;         // H = H_kv * group; group 1 is plain multi-head decode
   float scale_log2;        // scale * log2(e)
 };
 
@@ -85,14 +90,15 @@ __global__ void __launch_bounds__(DECODE_THREADS) sdpa_decode_split_kernel(const
   const int g = warp * GPW + lane / LPK;  // key group id
   const int e0 = (lane % LPK) * 8;        // first of this lane's 8 dimensions
   const size_t bh = (size_t)b * p.H + h;
+  const size_t bkv = (size_t)b * p.H_kv + h / p.group;  // the key/value head this query head reads
 
   float q[8];
   bf16x8_to_f32(*reinterpret_cast<const uint4*>(p.Q + bh * D + e0), q);
 #pragma unroll
   for (int i = 0; i < 8; ++i) q[i] *= p.scale_log2;
 
-  const __nv_bfloat16* Kb = p.K + bh * (size_t)p.n_cap * D + e0;
-  const __nv_bfloat16* Vb = p.V + bh * (size_t)p.n_cap * D + e0;
+  const __nv_bfloat16* Kb = p.K + bkv * (size_t)p.n_cap * D + e0;
+  const __nv_bfloat16* Vb = p.V + bkv * (size_t)p.n_cap * D + e0;
   const float NEG_INF = -__int_as_float(0x7f800000);
   float m = NEG_INF, l = 0.f, acc[8];
 #pragma unroll

@@ -58,8 +58,8 @@ struct PrefillCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
-  // q_full, full[NSLOT], empty[NSLOT], s_full[2], s_free[2], p_full[2], pv_done[2], o_full[2], turn[2], drain[2]
-  static constexpr int NBAR = 1 + 2 * NSLOT + 2 * 7;
+  // q_full, full[NSLOT], empty[NSLOT], s_full[2], s_free[2], p_full[2], pv_done[2], o_full[2], drain[2], turn[8]
+  static constexpr int NBAR = 1 + 2 * NSLOT + 2 * 6 + 8;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;  // + tmem slot, abort flag, align slack
   static constexpr int THREADS = 384;
   static constexpr int SOFTMAX_REGS = 216;
@@ -110,6 +110,9 @@ __host__ __device__ inline void prefill_kv_range(int r0, int n_q, int n_kv, int 
 #endif
 #ifndef SDPA_SM_TURN
 #define SDPA_SM_TURN 1
+#endif
+#ifndef SDPA_SM_TURN_WARP
+#define SDPA_SM_TURN_WARP 1
 #endif
 
 // Two finite, non-negative floats -> bf16x2 (lo in bits 0..15), rounded to nearest.
@@ -173,8 +176,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* p_full = s_free + 2;
   uint64_t* pv_done = p_full + 2;
   uint64_t* o_full = pv_done + 2;
-  uint64_t* turn = o_full + 2;
-  uint64_t* drain = turn + 2;
+  uint64_t* drain = o_full + 2;
+  uint64_t* turn = drain + 2;  // [query tile][warp within the warpgroup]
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -206,12 +209,12 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&s_full[x], 1);
       mbar_init(&s_free[x], 128);
       mbar_init(&p_full[x], 128);
-      mbar_init(&turn[x], 128);
       mbar_init(&pv_done[x], 1);
       mbar_init(&o_full[x], 1);
     }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    for (int w = 0; w < 8; ++w) mbar_init(&turn[w], SDPA_SM_TURN_WARP ? 32 : 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -378,14 +381,18 @@ __global__ void __launch_bounds__(384, 1)
     // that one's TMEM traffic, row maxima and hand-offs -- and, with P aliasing S, its
     // P V and next S MMAs -- overlap the other's exponentials.  Round j is tile a's turn,
     // then tile b's; both run T = max(ta, tb) rounds (a round without a tile only passes
-    // the turn).  turn[x] completes phase j when the other warpgroup hands over; tile b
-    // hands tile a its first turn up front.
-    if (SDPA_SM_TURN && x == 1) mbar_arrive(&turn[0]);
+    // the turn).  MUFU units belong to SM sub-partitions, and warp w of each warpgroup
+    // runs on sub-partition w, so the turn passes between those two warps alone
+    // (SDPA_SM_TURN_WARP) rather than between whole warpgroups.  my_turn completes phase
+    // j when the other warp hands over; tile b hands tile a its first turn up front.
+    uint64_t* my_turn = &turn[SDPA_SM_TURN_WARP ? 4 * x + (warp & 3) : 4 * x];
+    uint64_t* their_turn = &turn[SDPA_SM_TURN_WARP ? 4 * (x ^ 1) + (warp & 3) : 4 * (x ^ 1)];
+    if (SDPA_SM_TURN && x == 1) mbar_arrive(their_turn);
     for (int j = 0; ok && j < T; ++j) {
       if (j >= tiles) {  // no key tile left for this query tile: only pass the turn
         if (SDPA_SM_TURN) {
-          if (!(ok = wait_warp(&turn[x], j))) break;
-          mbar_arrive(&turn[x ^ 1]);
+          if (!(ok = wait_warp(my_turn, j))) break;
+          mbar_arrive(their_turn);
         }
         continue;
       }
@@ -448,11 +455,11 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      if (SDPA_SM_TURN && !(ok = wait_warp(&turn[x], j))) break;  // this warpgroup's turn on the exponentials
+      if (SDPA_SM_TURN && !(ok = wait_warp(my_turn, j))) break;  // this warp's turn on the exponentials
       const float m_use = (m_u == NEG_INF) ? 0.f : m_u;
       uint32_t pk[64];
       l += masked ? softmax_exp_row<false>(s, c2, m_use, pk) : softmax_exp_row<true>(s, c2, m_use, pk);
-      if (SDPA_SM_TURN) mbar_arrive(&turn[x ^ 1]);  // hand the exponentials over
+      if (SDPA_SM_TURN) mbar_arrive(their_turn);  // hand the exponentials over
       if (C::P_SEPARATE && j > 0 && !pv_waited) {  // P_x V of tile j-1 still reads P_x
         if (!(ok = wait_warp(&pv_done[x], j - 1))) break;
         tc_fence_after_sync();

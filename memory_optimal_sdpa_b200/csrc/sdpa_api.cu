@@ -14,6 +14,8 @@
 #include "prefill_bf16.cuh"
 #include "prefill_f32.cuh"
 #include "decode.cuh"
+#include "decode_gqa.cuh"
+#include "backward.cuh"
 
 namespace {
 
@@ -51,13 +53,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [bh][n][d] bf16 tensor, 64-column x 128-row boxes, 128-byte swizzle, zero fill out of bounds.
-bool make_map(CUtensorMap* map, const void* ptr, int d, int n, int bh) {
+// [bh][n][d] bf16 tensor, 64-column x box_rows-row boxes, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* ptr, int d, int n, int bh, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)bh};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -224,6 +226,8 @@ extern "C" int sdpa_decode(const void* Q, const void* K, const void* V, const in
   p.V = (const __nv_bfloat16*)V;
   p.kv_lens = kv_lens;
   p.H = heads;
+  p.H_kv = heads;
+  p.group = 1;
   p.n_cap = n_kv_cap;
   p.chunk = sdpa::decode_chunk(batch, heads, n_kv_cap);
   p.n_split = (n_kv_cap + p.chunk - 1) / p.chunk;
@@ -312,6 +316,8 @@ extern "C" int sdpa_decode_noalloc(const void* Q, const void* K, const void* V, 
   p.V = (const __nv_bfloat16*)V;
   p.kv_lens = kv_lens;
   p.H = heads;
+  p.H_kv = heads;
+  p.group = 1;
   p.n_cap = n_kv_cap;
   p.chunk = (int)chunk;
   p.n_split = (int)((n_kv_cap + chunk - 1) / chunk);
@@ -331,6 +337,197 @@ extern "C" int sdpa_decode_noalloc(const void* Q, const void* K, const void* V, 
   }
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SDPA_OK : cuda_fail("decode launch (static scratch)", e);
+}
+
+// ------------------------------------------------------------------ sdpa_decode_gqa
+namespace {
+// The tensor-core kernel takes d = 128 and groups of 2 .. 32 query heads; every other shape
+// runs the CUDA-core split kernel with its group mapping.
+bool gqa_tensor_path(int group, int d) { return d == 128 && group >= 2 && group <= 32; }
+
+long long gqa_chunk_for(long long batch, long long heads_q, long long heads_kv, long long n_cap, int d) {
+  return gqa_tensor_path((int)(heads_q / heads_kv), d) ? sdpa::gqa_chunk(batch, heads_kv, n_cap)
+                                                        : sdpa::decode_chunk(batch, heads_q, n_cap);
+}
+
+size_t gqa_ws_bytes(long long batch, long long heads_q, long long heads_kv, long long n_cap, long long d_v) {
+  const long long chunk = gqa_chunk_for(batch, heads_q, heads_kv, n_cap, (int)d_v);
+  const long long n_split = (n_cap + chunk - 1) / chunk;
+  return (size_t)(batch * heads_q * n_split * (d_v + 1)) * sizeof(float);
+}
+
+template <int NQ>
+int launch_decode_gqa(const void* Q, const void* K, const void* V, const int* kv_lens, float* part_o,
+                      float* part_lse, int batch, int heads_q, int heads_kv, int n_cap, int chunk, int n_split,
+                      float scale, cudaStream_t stream) {
+  using Cfg = sdpa::GqaCfg<NQ>;
+  auto kern = sdpa::sdpa_decode_gqa_kernel<NQ>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem, gqa)", attr_err);
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, 128, batch * heads_q, 1, NQ) || !make_map(&mk, K, 128, n_cap, batch * heads_kv) ||
+      !make_map(&mv, V, 128, n_cap, batch * heads_kv))
+    return SDPA_ERR_CUDA;
+  sdpa::GqaParams p;
+  p.part_o = part_o;
+  p.part_lse = part_lse;
+  p.kv_lens = kv_lens;
+  p.H_q = heads_q;
+  p.H_kv = heads_kv;
+  p.group = heads_q / heads_kv;
+  p.n_cap = n_cap;
+  p.chunk = chunk;
+  p.n_split = n_split;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  dim3 grid((unsigned)n_split, (unsigned)heads_kv, (unsigned)batch);
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SDPA_OK : cuda_fail("gqa decode launch", e);
+}
+}  // namespace
+
+extern "C" size_t sdpa_decode_gqa_workspace_size(int batch, int heads_q, int heads_kv, int n_kv_cap, int d_v) {
+  if (batch <= 0 || heads_q <= 0 || heads_kv <= 0 || heads_q % heads_kv != 0 || n_kv_cap <= 0 || d_v <= 0)
+    return 0;
+  return gqa_ws_bytes(batch, heads_q, heads_kv, n_kv_cap, d_v);
+}
+
+extern "C" int sdpa_decode_gqa(const void* Q, const void* K, const void* V, const int* kv_lens, void* O,
+                               float* LSE, int batch, int heads_q, int heads_kv, int n_kv_cap, int d_k, int d_v,
+                               float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (batch < 0 || heads_q < 0 || heads_kv < 1 || n_kv_cap < 1 || !std::isfinite(scale))
+    return SDPA_ERR_INVALID_ARG;
+  if (heads_q % heads_kv != 0) return SDPA_ERR_INVALID_ARG;
+  if (d_k != d_v || (d_k != 64 && d_k != 128)) return SDPA_ERR_UNSUPPORTED;
+  if (batch == 0 || heads_q == 0) return SDPA_OK;
+  if (!Q || !K || !V || !kv_lens || !O) return SDPA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned4(kv_lens) ||
+      (LSE && !aligned4(LSE)))
+    return SDPA_ERR_MISALIGNED;
+  if (batch > 65535 || heads_q > 65535) return SDPA_ERR_UNSUPPORTED;
+  if ((long long)batch * heads_q >= (1LL << 31) || (long long)batch * heads_kv * n_kv_cap >= (1LL << 31))
+    return SDPA_ERR_UNSUPPORTED;
+  const size_t need = gqa_ws_bytes(batch, heads_q, heads_kv, n_kv_cap, d_v);
+  if (!workspace || workspace_bytes < need) return SDPA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SDPA_ERR_MISALIGNED;
+  if (int e = check_device()) return e;
+  const int group = heads_q / heads_kv;
+  const int chunk = (int)gqa_chunk_for(batch, heads_q, heads_kv, n_kv_cap, d_k);
+  sdpa::DecodeParams p;  // the combine (and the CUDA-core split) parameters
+  p.Q = (const __nv_bfloat16*)Q;
+  p.K = (const __nv_bfloat16*)K;
+  p.V = (const __nv_bfloat16*)V;
+  p.kv_lens = kv_lens;
+  p.H = heads_q;
+  p.H_kv = heads_kv;
+  p.group = group;
+  p.n_cap = n_kv_cap;
+  p.chunk = chunk;
+  p.n_split = (n_kv_cap + chunk - 1) / chunk;
+  p.part_o = (float*)workspace;
+  p.part_lse = p.part_o + (size_t)batch * heads_q * p.n_split * d_v;
+  p.O = (__nv_bfloat16*)O;
+  p.LSE = LSE;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (gqa_tensor_path(group, d_k)) {
+    const int rc = group <= 16
+                       ? launch_decode_gqa<16>(Q, K, V, kv_lens, p.part_o, p.part_lse, batch, heads_q, heads_kv,
+                                               n_kv_cap, chunk, p.n_split, scale, s)
+                       : launch_decode_gqa<32>(Q, K, V, kv_lens, p.part_o, p.part_lse, batch, heads_q, heads_kv,
+                                               n_kv_cap, chunk, p.n_split, scale, s);
+    if (rc != SDPA_OK) return rc;
+    sdpa::sdpa_decode_combine_kernel<128><<<(unsigned)(batch * heads_q), 128, 0, s>>>(p);
+  } else {
+    dim3 grid((unsigned)p.n_split, (unsigned)heads_q, (unsigned)batch);
+    if (d_k == 64) {
+      sdpa::sdpa_decode_split_kernel<64><<<grid, sdpa::DECODE_THREADS, 0, s>>>(p);
+      sdpa::sdpa_decode_combine_kernel<64><<<(unsigned)(batch * heads_q), 64, 0, s>>>(p);
+    } else {
+      sdpa::sdpa_decode_split_kernel<128><<<grid, sdpa::DECODE_THREADS, 0, s>>>(p);
+      sdpa::sdpa_decode_combine_kernel<128><<<(unsigned)(batch * heads_q), 128, 0, s>>>(p);
+    }
+  }
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SDPA_OK : cuda_fail("gqa decode launch", e);
+}
+
+// ------------------------------------------------------------------ sdpa_bwd
+namespace {
+long long bwd_rows_padded(long long n_q) { return (n_q + 127) / 128 * 128; }
+
+template <int D, bool CAUSAL>
+int launch_bwd(const void* Q, const void* K, const void* V, const sdpa::BwdParams& p, cudaStream_t stream) {
+  using Cfg = sdpa::BwdCfg<D>;
+  auto kdkdv = sdpa::sdpa_bwd_dkdv_kernel<D, CAUSAL>;
+  auto kdq = sdpa::sdpa_bwd_dq_kernel<D, CAUSAL>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem, backward)", attr_err);
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, Q, D, p.n_q, p.bh_count) || !make_map(&mk, K, D, p.n_kv, p.bh_count) ||
+      !make_map(&mv, V, D, p.n_kv, p.bh_count) || !make_map(&mdo, p.dO, D, p.n_q, p.bh_count))
+    return SDPA_ERR_CUDA;
+  sdpa::sdpa_bwd_pre_kernel<D><<<dim3((unsigned)(p.n_q_pad / 128), (unsigned)p.bh_count), 128, 0, stream>>>(p);
+  const long long n_kt = (p.n_kv + 127) / 128, n_qt = (p.n_q + 127) / 128;
+  kdkdv<<<(unsigned)(p.bh_count * n_kt), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
+  kdq<<<(unsigned)(p.bh_count * n_qt), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SDPA_OK : cuda_fail("backward launch", e);
+}
+}  // namespace
+
+extern "C" size_t sdpa_bwd_workspace_size(int batch, int heads, int n_q) {
+  if (batch <= 0 || heads <= 0 || n_q <= 0) return 0;
+  return (size_t)(2LL * batch * heads * bwd_rows_padded(n_q)) * sizeof(float);
+}
+
+extern "C" int sdpa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                        void* dQ, void* dK, void* dV, int batch, int heads, int n_q, int n_kv, int d_k, int d_v,
+                        float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  if (batch < 0 || heads < 0 || n_q < 0 || n_kv < 1 || !std::isfinite(scale)) return SDPA_ERR_INVALID_ARG;
+  if (d_k != d_v || (d_k != 64 && d_k != 128) || !(scale > 0.f)) return SDPA_ERR_UNSUPPORTED;
+  if (batch == 0 || heads == 0 || n_q == 0) return SDPA_OK;
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return SDPA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned4(LSE) ||
+      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+    return SDPA_ERR_MISALIGNED;
+  const long long bh = (long long)batch * heads;
+  if (bh * (long long)(n_q > n_kv ? n_q : n_kv) >= (1LL << 31) || bh * ((n_kv + 127) / 128) >= (1LL << 31) ||
+      bh * bwd_rows_padded(n_q) >= (1LL << 31))
+    return SDPA_ERR_UNSUPPORTED;
+  const size_t need = sdpa_bwd_workspace_size(batch, heads, n_q);
+  if (!workspace || workspace_bytes < need) return SDPA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SDPA_ERR_MISALIGNED;
+  if (int e = check_device()) return e;
+  sdpa::BwdParams p;
+  p.O = (const __nv_bfloat16*)O;
+  p.dO = (const __nv_bfloat16*)dO;
+  p.LSE = LSE;
+  p.n_q = n_q;
+  p.n_kv = n_kv;
+  p.n_q_pad = (int)bwd_rows_padded(n_q);
+  p.bh_count = (int)bh;
+  p.Dvec = (float*)workspace;
+  p.L2 = p.Dvec + (size_t)bh * p.n_q_pad;
+  p.dQ = (__nv_bfloat16*)dQ;
+  p.dK = (__nv_bfloat16*)dK;
+  p.dV = (__nv_bfloat16*)dV;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (d_k == 64)
+    return causal ? launch_bwd<64, true>(Q, K, V, p, s) : launch_bwd<64, false>(Q, K, V, p, s);
+  return causal ? launch_bwd<128, true>(Q, K, V, p, s) : launch_bwd<128, false>(Q, K, V, p, s);
 }
 
 extern "C" int sdpa_get_last_device_error(void* stream) {

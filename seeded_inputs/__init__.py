@@ -19,6 +19,7 @@ from . import build as _build
 NORMAL = 0
 UNIFORM = 1
 STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_ROWS = 0, 1, 2, 3, 4
+STREAM_DO = 5  # the loss gradient dO of the backward pass
 
 _host = None
 _cuda = None

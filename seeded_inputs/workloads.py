@@ -6,6 +6,7 @@
   cfg4  bf16 prefill, B=1 H=8 n=32768 d=128, Q,K ~ N(0, 2.5^2), V ~ N(0,1), scale 1/sqrt(128), non-causal
   cfg5  bf16 decode, B=64 H=32 n_cap=16384 d=128, lengths ~ U{1024..16384}, N(0,1), scale 1/sqrt(128)
   cfg3w cfg3 with a causal local window of 512 keys (window_left = 511, window_right = 0)
+  cfg5g cfg5 with grouped-query heads: 64 query heads over 8 key/value heads (groups of 8)
 
 Streams: Q = 0, K = 1, V = 2 (counter = flat element index of the tensor), decode
 lengths = 3, sampled rows = 4.  Seed 0 everywhere.  bf16 values are the RNE
@@ -76,13 +77,18 @@ class Prefill:
 class Decode:
     name: str
     batch: int
-    heads: int
+    heads: int      # query heads
     n_cap: int
     d: int
     len_lo: int
     len_hi: int
     scale: float
     seed: int = 0
+    heads_kv: int = 0  # key/value heads (0: one per query head)
+
+    @property
+    def kv_heads(self):
+        return self.heads_kv or self.heads
 
     @property
     def scale_f32(self):
@@ -94,7 +100,7 @@ class Decode:
     def bytes(self, lens=None):
         """Algorithmic bytes: the valid K and V rows, Q, O and LSE (bf16 except LSE)."""
         lens = self.lengths() if lens is None else lens
-        kv = int(np.sum(lens, dtype=np.int64)) * self.heads * self.d * 2 * 2
+        kv = int(np.sum(lens, dtype=np.int64)) * self.kv_heads * self.d * 2 * 2
         return kv + self.batch * self.heads * (self.d * 2 * 2 + 4)
 
     def flops(self, lens=None):
@@ -113,6 +119,8 @@ CFG4 = Prefill("cfg4", 1, 8, 32768, 32768, 128, False, "bf16", 1 / 128 ** 0.5, q
 CFG3W = Prefill("cfg3w", 1, 32, 8192, 8192, 128, True, "bf16", 1 / 128 ** 0.5, v=Dist(UNIFORM, -1.0, 1.0),
                 window=(511, 0))
 CFG5 = Decode("cfg5", 64, 32, 16384, 128, 1024, 16384, 1 / 128 ** 0.5)
+# cfg5's batch, cache and lengths with 64 query heads over 8 key/value heads (groups of 8)
+CFG5G = Decode("cfg5g", 64, 64, 16384, 128, 1024, 16384, 1 / 128 ** 0.5, heads_kv=8)
 
 
 def prefill_host(w):

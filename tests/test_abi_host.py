@@ -28,7 +28,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
-        "sdpa_decode", "sdpa_decode_noalloc", "sdpa_decode_workspace_size", "sdpa_fwd", "sdpa_fwd_f32",
+        "sdpa_bwd", "sdpa_bwd_workspace_size", "sdpa_decode", "sdpa_decode_gqa", "sdpa_decode_gqa_workspace_size", "sdpa_decode_noalloc",
+        "sdpa_decode_workspace_size", "sdpa_fwd", "sdpa_fwd_f32",
         "sdpa_fwd_window",
         "sdpa_get_last_device_error", "sdpa_status_string"])
 
@@ -118,6 +119,52 @@ def test_decode_workspace_and_errors(sdpa):
     assert call(args(dk=80, dv=80)) == sdpa.SDPA_ERR_UNSUPPORTED
     assert call(args(V=P + 4)) == sdpa.SDPA_ERR_MISALIGNED
     assert call(args(b=0)) == sdpa.SDPA_OK
+
+
+def test_decode_gqa_workspace_and_errors(sdpa):
+    ws = sdpa.decode_gqa_workspace_size
+    assert ws(0, 8, 1, 16, 128) == 0 and ws(1, 6, 4, 16, 128) == 0 and ws(1, 8, 0, 16, 128) == 0
+    # 64 batches x 64 query heads over 8 key/value heads, 16384-row cache, d = 128 (tensor-core
+    # path): 2048-key splits, 8 per head, each d_v + 1 floats per query head
+    assert ws(64, 64, 8, 16384, 128) == 64 * 64 * 8 * 129 * 4
+    # group size one is plain decode and sizes like it
+    assert ws(64, 32, 32, 16384, 128) == sdpa.decode_workspace_size(64, 32, 16384, 128)
+    d = sdpa.lib.sdpa_decode_gqa
+    need = ws(2, 8, 2, 256, 128)
+    args = lambda **kw: dict(dict(Q=P, K=P, V=P, L=P, O=P, LSE=None, b=2, hq=8, hkv=2, cap=256, dk=128, dv=128,
+                                  scale=0.1, ws=P, wsb=need), **kw)
+    call = lambda a: d(a["Q"], a["K"], a["V"], a["L"], a["O"], a["LSE"], a["b"], a["hq"], a["hkv"], a["cap"],
+                       a["dk"], a["dv"], a["scale"], a["ws"], a["wsb"], None)
+    assert call(args(ws=None)) == sdpa.SDPA_ERR_WORKSPACE
+    assert call(args(wsb=need - 1)) == sdpa.SDPA_ERR_WORKSPACE
+    assert call(args(hkv=3)) == sdpa.SDPA_ERR_INVALID_ARG
+    assert call(args(hkv=0)) == sdpa.SDPA_ERR_INVALID_ARG
+    assert call(args(L=None)) == sdpa.SDPA_ERR_INVALID_ARG
+    assert call(args(scale=float("nan"))) == sdpa.SDPA_ERR_INVALID_ARG
+    assert call(args(dk=96, dv=96)) == sdpa.SDPA_ERR_UNSUPPORTED
+    assert call(args(K=P + 8)) == sdpa.SDPA_ERR_MISALIGNED
+    assert call(args(b=0)) == sdpa.SDPA_OK and call(args(hq=0)) == sdpa.SDPA_OK
+
+
+def test_bwd_workspace_and_errors(sdpa):
+    ws = sdpa.bwd_workspace_size
+    assert ws(0, 1, 16) == 0 and ws(1, 1, 0) == 0
+    assert ws(4, 16, 2048) == 2 * 4 * 16 * 2048 * 4 and ws(1, 2, 130) == 2 * 2 * 256 * 4
+    d = sdpa.lib.sdpa_bwd
+    need = ws(1, 2, 256)
+    args = lambda **kw: dict(dict(Q=P, K=P, V=P, O=P, dO=P, L=P, dQ=P, dK=P, dV=P, b=1, h=2, nq=256, nkv=256, dk=64,
+                                  dv=64, scale=0.125, causal=1, ws=P, wsb=need), **kw)
+    call = lambda a: d(a["Q"], a["K"], a["V"], a["O"], a["dO"], a["L"], a["dQ"], a["dK"], a["dV"], a["b"], a["h"],
+                       a["nq"], a["nkv"], a["dk"], a["dv"], a["scale"], a["causal"], a["ws"], a["wsb"], None)
+    assert call(args(ws=None)) == sdpa.SDPA_ERR_WORKSPACE
+    assert call(args(wsb=need - 1)) == sdpa.SDPA_ERR_WORKSPACE
+    assert call(args(L=None)) == sdpa.SDPA_ERR_INVALID_ARG
+    assert call(args(dO=None)) == sdpa.SDPA_ERR_INVALID_ARG
+    assert call(args(nkv=0)) == sdpa.SDPA_ERR_INVALID_ARG
+    assert call(args(dk=128, dv=64)) == sdpa.SDPA_ERR_UNSUPPORTED
+    assert call(args(scale=-1.0)) == sdpa.SDPA_ERR_UNSUPPORTED
+    assert call(args(dQ=P + 2)) == sdpa.SDPA_ERR_MISALIGNED
+    assert call(args(nq=0)) == sdpa.SDPA_OK
 
 
 def test_status_strings(sdpa):

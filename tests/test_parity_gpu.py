@@ -223,6 +223,146 @@ def test_cfg3w_window_full_size_sampled(sdpa, cuda_device):
         check_bf16(O[0, h, rows], O_ref, L[0, h, rows], L_ref, "cfg3w h=%d" % h)
 
 
+# ------------------------------------------------------------------------------------ grouped-query decode
+GQA_CASES = [
+    # (B, H_q, H_kv, n_cap, d, lens)   groups of 2 .. 32 at d = 128 take the tensor cores
+    (3, 8, 4, 1000, 128, (1, 1000, 517)), (2, 16, 4, 3000, 128, (2049, 129)), (2, 16, 2, 2100, 128, (128, 2100)),
+    (1, 32, 2, 700, 128, (700,)), (2, 64, 2, 400, 128, (255, 400)), (1, 24, 2, 333, 128, (333,)),
+    (2, 40, 2, 260, 128, (1, 260)),
+    # other shapes: the CUDA-core kernel with the same head mapping
+    (1, 64, 1, 300, 128, (300,)), (2, 12, 3, 500, 64, (77, 500)), (2, 4, 4, 300, 128, (5, 300)),
+]
+
+
+def _to_bf16_bits(x):
+    """float32 -> bf16 bit patterns, round to nearest even (NaN -> the quiet NaN 0x7FC0)."""
+    u = np.ascontiguousarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    return np.where(np.isnan(x), np.uint16(0x7FC0), r)
+
+
+def _gqa_inputs(B, H_q, H_kv, n_cap, d, lens, seed):
+    q = si.fill_host((B, H_q, d), seed, 0)
+    k = si.fill_host((B, H_kv, n_cap, d), seed, 1)
+    v = si.fill_host((B, H_kv, n_cap, d), seed, 2)
+    for b in range(B):  # rows past the length hold NaN: any use of them poisons O
+        k[b, :, lens[b]:] = 0x7FC0
+        v[b, :, lens[b]:] = 0x7FC0
+    return q, k, v
+
+
+@pytest.mark.parametrize("B,H_q,H_kv,n_cap,d,lens", GQA_CASES)
+def test_decode_gqa_small_every_pair(sdpa, cuda_device, B, H_q, H_kv, n_cap, d, lens):
+    import torch
+    lens = np.array(lens, np.int32)
+    q, k, v = _gqa_inputs(B, H_q, H_kv, n_cap, d, lens, 11 + H_q + n_cap)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    _, tq = _bits_to_torch(q, cuda_device)
+    tk, tv = (W.to_torch(x, cuda_device) for x in (k, v))
+    tl = torch.from_numpy(lens).to(cuda_device)
+    o_flat, o = _nan_buffer((B, H_q, d), torch.bfloat16, cuda_device, 256)
+    l_flat, lse = _nan_buffer((B, H_q), torch.float32, cuda_device, 64)
+    sdpa.decode_gqa(tq, tk, tv, tl, scale=scale, o=o, lse=lse)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O_ref, L_ref = oracle.decode_gqa(*(si.bf16_bits_to_f32(x) for x in (q, k, v)), lens, scale)
+    check_bf16(o.float().cpu().numpy().reshape(B * H_q, d), O_ref, lse.cpu().numpy().reshape(-1), L_ref,
+               "gqa %s" % ((B, H_q, H_kv, n_cap, d, tuple(lens)),))
+    assert torch.isnan(o_flat[o.numel():]).all() and torch.isnan(l_flat[lse.numel():]).all()
+
+
+def test_decode_gqa_group_of_one_is_decode(sdpa, cuda_device):
+    import torch
+    B, H, n_cap, d = 2, 4, 600, 128
+    lens = np.array([600, 37], np.int32)
+    q, k, v = _gqa_inputs(B, H, H, n_cap, d, lens, 3)
+    tq, tk, tv = (W.to_torch(x, cuda_device) for x in (q, k, v))
+    tl = torch.from_numpy(lens).to(cuda_device)
+    o1, l1 = sdpa.decode_gqa(tq, tk, tv, tl)
+    o2, l2 = sdpa.decode(tq, tk, tv, tl)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def _gqa_medium(sdpa, device, q, k, v, lens, scale, what, n_groups=24):
+    """A cache large enough for several 128-key tiles per split; seeded (batch, group) samples."""
+    import torch
+    B, H_q, d = q.shape
+    H_kv, n_cap = k.shape[1], k.shape[2]
+    G = H_q // H_kv
+    tl = torch.from_numpy(lens).to(device)
+    o, lse = sdpa.decode_gqa(W.to_torch(q, device), W.to_torch(k, device), W.to_torch(v, device), tl, scale=scale)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O = o.float().cpu().numpy()
+    L = lse.cpu().numpy()
+    for bg in sorted(set(int(x) for x in si.sample_rows(B * H_kv, n_groups, 7, salt=5))):
+        b, kvh = divmod(bg, H_kv)
+        n = int(lens[b])
+        hs = slice(kvh * G, kvh * G + G)
+        O_ref, L_ref = oracle.decode_gqa(si.bf16_bits_to_f32(q[b:b + 1, hs]), si.bf16_bits_to_f32(k[b:b + 1, kvh:kvh + 1]),
+                                         si.bf16_bits_to_f32(v[b:b + 1, kvh:kvh + 1]), np.array([n], np.int32), scale)
+        check_bf16(O[b, hs], O_ref, L[b, hs], L_ref, "%s b=%d kv head %d len=%d" % (what, b, kvh, n))
+
+
+def test_decode_gqa_multi_tile_splits(sdpa, cuda_device):
+    # 32 x 2 key/value heads x 8192 rows: 512-key splits, four 128-key tiles each
+    B, H_q, H_kv, n_cap, d = 32, 16, 2, 8192, 128
+    assert sdpa.decode_gqa_workspace_size(B, H_q, H_kv, n_cap, d) == B * H_q * (n_cap // 512) * (d + 1) * 4
+    lens = si.kv_lengths(B, 1, n_cap, 21)
+    lens[:4] = (1, 511, 513, n_cap)
+    q, k, v = _gqa_inputs(B, H_q, H_kv, n_cap, d, lens, 21)
+    _gqa_medium(sdpa, cuda_device, q, k, v, lens, float(np.float32(1 / math.sqrt(d))), "gqa multi-tile")
+
+
+def test_decode_gqa_rescale_inside_a_split(sdpa, cuda_device):
+    # Scores that climb by ~12 (log2 units) from one 128-key tile to the next move every
+    # head's reference maximum inside a split; a negative scale is accepted here too.
+    B, H_q, H_kv, n_cap, d = 32, 16, 2, 8192, 128
+    lens = np.full(B, n_cap, np.int32)
+    lens[1::2] = si.kv_lengths(B // 2, 600, n_cap, 4)
+    q, k, v = _gqa_inputs(B, H_q, H_kv, n_cap, d, lens, 4)
+    qf = np.abs(si.bf16_bits_to_f32(q)) * 0.25 + 0.5
+    kf = si.bf16_bits_to_f32(k) * 0.05 + ((np.arange(n_cap) // 128) % 4 * 0.75)[None, None, :, None]
+    for sign in (1.0, -1.0):
+        q2 = _to_bf16_bits(qf)
+        k2 = _to_bf16_bits(kf)
+        _gqa_medium(sdpa, cuda_device, q2, k2, v, lens, sign * float(np.float32(1 / math.sqrt(d))),
+                    "gqa rescale sign %+d" % sign, n_groups=12)
+
+
+def test_cfg5g_decode_full_size_sampled(sdpa, cuda_device):
+    import torch
+    w = W.CFG5G
+    G = w.heads // w.kv_heads
+    lens = w.lengths()
+    tl = torch.from_numpy(lens).to(cuda_device)
+    shape = (w.batch, w.kv_heads, w.n_cap, w.d)
+    tk = torch.empty(shape, dtype=torch.bfloat16, device=cuda_device)
+    tv = torch.empty(shape, dtype=torch.bfloat16, device=cuda_device)
+    si.fill_device_cache(tk, tl, w.seed, si.STREAM_K)
+    si.fill_device_cache(tv, tl, w.seed, si.STREAM_V)
+    q = si.fill_host((w.batch, w.heads, w.d), w.seed, si.STREAM_Q)
+    o, lse = sdpa.decode_gqa(W.to_torch(q, cuda_device), tk, tv, tl, scale=w.scale_f32)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O = o.float().cpu().numpy()
+    L = lse.cpu().numpy()
+    del tk, tv
+    torch.cuda.empty_cache()
+    # (batch, key/value head) groups: the shortest and the longest sequence, plus seeded picks
+    b_min, b_max = int(np.argmin(lens)), int(np.argmax(lens))
+    picks = {b_min * w.kv_heads, b_max * w.kv_heads + w.kv_heads - 1}
+    picks |= set(int(x) for x in si.sample_rows(w.batch * w.kv_heads, 30, w.seed, salt=98))
+    for bg in sorted(picks):
+        b, kvh = divmod(bg, w.kv_heads)
+        n = int(lens[b])
+        start = ((b * w.kv_heads + kvh) * w.n_cap) * w.d
+        kf = si.bf16_bits_to_f32(si.fill_host((1, 1, n, w.d), w.seed, si.STREAM_K, start=start))
+        vf = si.bf16_bits_to_f32(si.fill_host((1, 1, n, w.d), w.seed, si.STREAM_V, start=start))
+        hs = slice(kvh * G, kvh * G + G)
+        O_ref, L_ref = oracle.decode_gqa(si.bf16_bits_to_f32(q[b:b + 1, hs]), kf, vf, np.array([n], np.int32),
+                                         w.scale_f32)
+        check_bf16(O[b, hs], O_ref, L[b, hs], L_ref, "cfg5g b=%d kv head %d len=%d" % (b, kvh, n))
+
+
 # ----------------------------------------------------------------------------------------------- fp32 path
 F32_CASES = [(1, 1, 128, 128, 64, 64, False), (1, 1, 128, 128, 64, 64, True), (2, 3, 77, 130, 33, 100, True),
              (1, 2, 200, 50, 128, 128, True), (1, 1, 1, 1, 1, 1, False), (1, 2, 65, 300, 3, 128, False)]
