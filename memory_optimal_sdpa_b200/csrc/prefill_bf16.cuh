@@ -417,12 +417,12 @@ __global__ void __launch_bounds__(384, 1)
           if (kv0 + c > lim || kv0 + c < lo) s[c] = __float_as_uint(NEG_INF);
       }
       float mx;
-      {  // eight independent chains of 3-input maxima
+      {  // eight independent chains of 3-input maxima over s[0..127]: 16 + 7 x 16 scores
         float m[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m[k] = __uint_as_float(s[k]);
+        for (int k = 0; k < 8; ++k) m[k] = fmaxf(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1]));
 #pragma unroll
-        for (int c = 8; c < 128; c += 16)
+        for (int c = 16; c < 128; c += 16)
 #pragma unroll
           for (int k = 0; k < 8; ++k) m[k] = max3f(m[k], __uint_as_float(s[c + 2 * k]), __uint_as_float(s[c + 2 * k + 1]));
         mx = max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));

@@ -99,6 +99,43 @@ def test_prefill_bf16_small(sdpa, cuda_device, B, H, n_q, n_kv, d, causal):
         assert (O[:, :, :n_q - n_kv] == 0).all()
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_causal_first_row_is_exact(sdpa, cuda_device, d):
+    # Causal row 0 (n_q = n_kv) sees key 0 alone: P = 1 exactly, so O[0] = V[0] bit for bit
+    # and LSE[0] = scale q_0 . k_0.  Any reference maximum above the row's true maximum (a
+    # score the row may not see, or a stray value) makes P < 1 and shows here.
+    import torch
+    B, H, n = 2, 8, 256
+    for seed in range(6):
+        q, k, v = (si.fill_host((B, H, n, d), 100 + seed, s_) for s_ in (0, 1, 2))
+        scale = float(np.float32(1 / math.sqrt(d)))
+        o, lse = sdpa.fwd(*(W.to_torch(x, cuda_device) for x in (q, k, v)), causal=True, scale=scale)
+        torch.cuda.synchronize()
+        O = o.float().cpu().numpy()
+        V = si.bf16_bits_to_f32(v)
+        assert np.array_equal(O[:, :, 0], V[:, :, 0]), "seed %d: row 0 differs from V[0] in %d places" % (
+            seed, int((O[:, :, 0] != V[:, :, 0]).sum()))
+        s00 = np.einsum("bhd,bhd->bh", si.bf16_bits_to_f32(q)[:, :, 0].astype(np.float64),
+                        si.bf16_bits_to_f32(k)[:, :, 0].astype(np.float64)) * scale
+        assert np.abs(lse.cpu().numpy()[:, :, 0] - s00).max() < 1e-5
+
+
+def test_prefill_identity_values_give_probabilities(sdpa, cuda_device):
+    # V = I (n_kv = d): O = P row by row, so every probability the kernel forms is visible;
+    # each entry is within two bf16 roundings (P, then O) of the exact softmax.
+    import torch
+    for d in (64, 128):
+        for causal in (False, True):
+            q, k = (si.fill_host((1, 2, d, d), 31, s_) for s_ in (0, 1))
+            v = np.broadcast_to(np.eye(d, dtype=np.float32), (1, 2, d, d)).copy()
+            scale = float(np.float32(1 / math.sqrt(d)))
+            o, _ = sdpa.fwd(*(W.to_torch(x, cuda_device) for x in (q, k)),
+                            torch.from_numpy(v).to(cuda_device).to(torch.bfloat16), causal=causal, scale=scale)
+            P, _ = oracle.sdpa_rows(si.bf16_bits_to_f32(q), si.bf16_bits_to_f32(k), v, scale, causal)
+            O = o.float().cpu().numpy()
+            assert (np.abs(O - P) <= 2 ** -7 * P + 1e-6).all(), "d=%d causal=%d" % (d, causal)
+
+
 def test_prefill_lse_optional_and_repeatable(sdpa, cuda_device):
     import torch
     B, H, n, d = 1, 4, 384, 128
