@@ -40,6 +40,7 @@ sys.path.insert(0, ROOT)
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_SOURCES = ["memory_optimal_sdpa_b200/csrc/prefill_bf16.cuh", "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
 DECODE_SOURCES = ["memory_optimal_sdpa_b200/csrc/decode.cuh"]
+BWD_SOURCES = ["memory_optimal_sdpa_b200/csrc/backward.cuh", "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
 GQA_SOURCES = ["memory_optimal_sdpa_b200/csrc/decode_gqa.cuh", "memory_optimal_sdpa_b200/csrc/decode.cuh",
                "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
 
@@ -426,7 +427,10 @@ def run_backward(args, sdpa, si, W, works, q, k, v, outs, stream, flush, peaks, 
                                     "achieved": round(flops / t / 1e12, 1), "peak": peak, "unit": "TFLOP/s",
                                     "frac": round(flops / t / 1e12 / peak, 4),
                                     "peak_kind": peak_kind + " burst bf16", "algorithmic_flop": flops,
-                                    "executed_flop": 3.5 * w.flops(), "traffic": None}}
+                                    "executed_flop": 3.5 * w.flops(),
+                                    "traffic": (profiled_traffic("backward_cfg2_dram.txt", BWD_SOURCES)
+                                                if w.name == "cfg2" else None),
+                                    "traffic_covers": "dK/dV and dQ kernels (ncu); not the preprocess kernel"}}
     del dq, dk, dv, ws, do
     return res
 
