@@ -56,8 +56,8 @@ struct BwdCfg {
   static constexpr int FIX_OFF = 0;                // the CTA's fixed pair: (K, V) or (Q, dO)
   static constexpr int ST_OFF = 2 * TILE_BYTES;    // streamed stages: (Q, dO, vectors) or (K, V)
   static constexpr int BAR_OFF = ST_OFF + NSTAGE * STAGE_BYTES;
-  // fix_full, full[NSTAGE], empty[NSTAGE], s_full, p_full[2], o_full, drain
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 5;
+  // fix_full, full[NSTAGE], empty[NSTAGE], s_full[2], p_full[2], o_full, drain
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 6;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;
   static constexpr int THREADS = 384;
   static constexpr int EW_REGS = 216;
@@ -154,8 +154,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* fix_full = bars;
   uint64_t* full = bars + 1;
   uint64_t* empty = full + C::NSTAGE;
-  uint64_t* s_full = empty + C::NSTAGE;
-  uint64_t* p_full = s_full + 1;  // [warpgroup]
+  uint64_t* s_full = empty + C::NSTAGE;  // [half]
+  uint64_t* p_full = s_full + 2;         // [half] = [warpgroup]
   uint64_t* o_full = p_full + 2;
   uint64_t* drain = o_full + 1;
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
@@ -181,7 +181,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(&p_full[0], 128);
     mbar_init(&p_full[1], 128);
     mbar_init(o_full, 1);
@@ -237,42 +238,57 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == C::MMA_WARP) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0 && NT > 0) {
-        constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // K or V (K-major) x Q or dO (K-major)
-        constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);     // P^T or dS^T (TMEM) x dO or Q (MN-major)
+        constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);  // K or V (K-major) x 64 rows of Q or dO
+        constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);    // P^T or dS^T (TMEM) x dO or Q (MN-major)
         const uint32_t fix = smem_u32(sFix), st0 = smem_u32(sSt);
         const uint64_t dK = smem_desc_sw128(fix, 16, 1024);
         const uint64_t dV = smem_desc_sw128(fix + C::TILE_BYTES, 16, 1024);
         auto wait_bar = [&](uint64_t* bar, int phase) {
           return mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
         };
-        bool ok = wait_bar(fix_full, 0);
-        for (int t = 0; ok && t < NT; ++t) {
-          const int st = t % C::NSTAGE;
-          const uint32_t sq = st0 + st * C::STAGE_BYTES, sdo = sq + C::TILE_BYTES;
-          if (!(ok = wait_bar(&full[st], t / C::NSTAGE))) break;
-          const uint64_t dQk = smem_desc_sw128(sq, 16, 1024), dOk = smem_desc_sw128(sdo, 16, 1024);
+        // Query tile t is taken in two halves of 64 rows; half h's S^T and dP^T go to columns
+        // [64 h, 64 h + 64) of their regions, where warpgroup h reads them.
+        auto issue_sdp = [&](int t, int h) {  // S^T_h = K Q_h^T, dP^T_h = V dO_h^T
+          const uint32_t sq = st0 + (t % C::NSTAGE) * C::STAGE_BYTES + h * 8192;  // 64 rows in
+          const uint64_t dQk = smem_desc_sw128(sq, 16, 1024), dOk = smem_desc_sw128(sq + C::TILE_BYTES, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K Q^T, dP^T = V dO^T
+          for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t o = (uint64_t)((((kk >> 2) * C::BLOCK_BYTES) + (kk & 3) * 32) >> 4);
-            mma_ss(tmem + C::COL_S, dK + o, dQk + o, idS, kk > 0 ? 1u : 0u);
-            mma_ss(tmem + C::COL_DP, dV + o, dOk + o, idS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_S + 64 * h, dK + o, dQk + o, idS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_DP + 64 * h, dV + o, dOk + o, idS, kk > 0 ? 1u : 0u);
           }
-          tc_commit(s_full);
-          const uint64_t dOm = smem_desc_sw128(sdo, C::BLOCK_BYTES, 1024);  // MN-major views
+          tc_commit(&s_full[h]);
+        };
+        auto issue_grad = [&](int t, int h) {  // dV += P^T_h dO_h, dK += dS^T_h Q_h (64 query rows)
+          const uint32_t sq = st0 + (t % C::NSTAGE) * C::STAGE_BYTES;
+          const uint64_t dOm = smem_desc_sw128(sq + C::TILE_BYTES, C::BLOCK_BYTES, 1024);  // MN-major views
           const uint64_t dQm = smem_desc_sw128(sq, C::BLOCK_BYTES, 1024);
-          for (int w = 0; ok && w < 2; ++w) {  // each warpgroup's 64 query columns as soon as they are ready
-            if (!(ok = wait_bar(&p_full[w], t))) break;
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              const int kk = 4 * w + k4;
-              const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-              const uint64_t ob = (uint64_t)((kk * 2048) >> 4);
-              mma_ts(tmem + C::COL_A, tmem + C::COL_S + bwd_pair_col(kk), dOm + ob, idA, acc);   // dV += P^T dO
-              mma_ts(tmem + C::COL_B, tmem + C::COL_DP + bwd_pair_col(kk), dQm + ob, idA, acc);  // dK += dS^T Q
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = 4 * h + k4;
+            const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t ob = (uint64_t)((kk * 2048) >> 4);
+            mma_ts(tmem + C::COL_A, tmem + C::COL_S + bwd_pair_col(kk), dOm + ob, idA, acc);
+            mma_ts(tmem + C::COL_B, tmem + C::COL_DP + bwd_pair_col(kk), dQm + ob, idA, acc);
+          }
+        };
+        // Half h of tile t + 1 starts as soon as warpgroup h has finished half h of tile t, so one
+        // warpgroup's elementwise pass overlaps the other's and the tensor core's products.
+        bool ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0);
+        if (ok) {
+          issue_sdp(0, 0);
+          issue_sdp(0, 1);
+        }
+        for (int t = 0; ok && t < NT; ++t) {
+          for (int h = 0; ok && h < 2; ++h) {
+            if (!(ok = wait_bar(&p_full[h], t))) break;
+            issue_grad(t, h);
+            if (h == 1) tc_commit(&empty[t % C::NSTAGE]);
+            if (t + 1 < NT) {
+              if (h == 0 && !(ok = wait_bar(&full[(t + 1) % C::NSTAGE], (t + 1) / C::NSTAGE))) break;
+              issue_sdp(t + 1, h);
             }
           }
-          if (!ok) break;
-          tc_commit(&empty[st]);
         }
         if (ok) tc_commit(o_full);
         tc_commit(drain);
@@ -297,7 +313,7 @@ __global__ void __launch_bounds__(384, 1)
       const float* vL2 = reinterpret_cast<const float*>(sSt + st * C::STAGE_BYTES + 2 * C::TILE_BYTES);
       const float* vD = vL2 + 128;
       // the stage's vectors come from the bulk copy: wait for it here too, not only through the MMAs
-      if (!(ok = wait_warp(&full[st], t / C::NSTAGE) && wait_warp(s_full, t))) break;
+      if (!(ok = wait_warp(&full[st], t / C::NSTAGE) && wait_warp(&s_full[w], t))) break;
       tc_fence_after_sync();
       const int q0 = (t_first + t) * 128 + 64 * w;  // first query of this warpgroup's columns
       const bool masked = CAUSAL && (q0 + off < j0 + 127);
@@ -384,8 +400,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* fix_full = bars;
   uint64_t* full = bars + 1;
   uint64_t* empty = full + C::NSTAGE;
-  uint64_t* s_full = empty + C::NSTAGE;
-  uint64_t* p_full = s_full + 1;
+  uint64_t* s_full = empty + C::NSTAGE;  // [half]
+  uint64_t* p_full = s_full + 2;         // [half] = [warpgroup]
   uint64_t* o_full = p_full + 2;
   uint64_t* drain = o_full + 1;
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
@@ -410,7 +426,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(&p_full[0], 128);
     mbar_init(&p_full[1], 128);
     mbar_init(o_full, 1);
@@ -462,39 +479,49 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == C::MMA_WARP) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0 && T > 0) {
-        constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q or dO (K-major) x K or V (K-major)
-        constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);     // dS (TMEM) x K (MN-major)
+        constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);  // Q or dO (K-major) x 64 rows of K or V
+        constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);    // dS (TMEM) x K (MN-major)
         const uint32_t fix = smem_u32(sFix), st0 = smem_u32(sSt);
         const uint64_t dQk = smem_desc_sw128(fix, 16, 1024);
         const uint64_t dOk = smem_desc_sw128(fix + C::TILE_BYTES, 16, 1024);
         auto wait_bar = [&](uint64_t* bar, int phase) {
           return mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
         };
-        bool ok = wait_bar(fix_full, 0);
-        for (int j = 0; ok && j < T; ++j) {
-          const int st = j % C::NSTAGE;
-          const uint32_t sk = st0 + st * C::STAGE_BYTES, sv = sk + C::TILE_BYTES;
-          if (!(ok = wait_bar(&full[st], j / C::NSTAGE))) break;
-          const uint64_t dKk = smem_desc_sw128(sk, 16, 1024), dVk = smem_desc_sw128(sv, 16, 1024);
+        auto issue_sdp = [&](int j, int h) {  // S_h = Q K_h^T, dP_h = dO V_h^T (64 keys)
+          const uint32_t sk = st0 + (j % C::NSTAGE) * C::STAGE_BYTES + h * 8192;
+          const uint64_t dKk = smem_desc_sw128(sk, 16, 1024), dVk = smem_desc_sw128(sk + C::TILE_BYTES, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {  // S = Q K^T, dP = dO V^T
+          for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t o = (uint64_t)((((kk >> 2) * C::BLOCK_BYTES) + (kk & 3) * 32) >> 4);
-            mma_ss(tmem + C::COL_S, dQk + o, dKk + o, idS, kk > 0 ? 1u : 0u);
-            mma_ss(tmem + C::COL_DP, dOk + o, dVk + o, idS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_S + 64 * h, dQk + o, dKk + o, idS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_DP + 64 * h, dOk + o, dVk + o, idS, kk > 0 ? 1u : 0u);
           }
-          tc_commit(s_full);
-          const uint64_t dKm = smem_desc_sw128(sk, C::BLOCK_BYTES, 1024);
-          for (int w = 0; ok && w < 2; ++w) {
-            if (!(ok = wait_bar(&p_full[w], j))) break;
+          tc_commit(&s_full[h]);
+        };
+        auto issue_grad = [&](int j, int h) {  // dQ += dS_h K_h
+          const uint64_t dKm = smem_desc_sw128(st0 + (j % C::NSTAGE) * C::STAGE_BYTES, C::BLOCK_BYTES, 1024);
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              const int kk = 4 * w + k4;
-              mma_ts(tmem + C::COL_A, tmem + C::COL_DP + bwd_pair_col(kk), dKm + (uint64_t)((kk * 2048) >> 4), idA,
-                     (j > 0 || kk > 0) ? 1u : 0u);  // dQ += dS K
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = 4 * h + k4;
+            mma_ts(tmem + C::COL_A, tmem + C::COL_DP + bwd_pair_col(kk), dKm + (uint64_t)((kk * 2048) >> 4), idA,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          }
+        };
+        bool ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0);
+        if (ok) {
+          issue_sdp(0, 0);
+          issue_sdp(0, 1);
+        }
+        for (int j = 0; ok && j < T; ++j) {
+          for (int h = 0; ok && h < 2; ++h) {
+            if (!(ok = wait_bar(&p_full[h], j))) break;
+            issue_grad(j, h);
+            if (h == 1) tc_commit(&empty[j % C::NSTAGE]);
+            if (j + 1 < T) {
+              if (h == 0 && !(ok = wait_bar(&full[(j + 1) % C::NSTAGE], (j + 1) / C::NSTAGE))) break;
+              issue_sdp(j + 1, h);
             }
           }
-          if (!ok) break;
-          tc_commit(&empty[st]);
         }
         if (ok) tc_commit(o_full);
         tc_commit(drain);
@@ -518,7 +545,7 @@ __global__ void __launch_bounds__(384, 1)
       return __all_sync(0xffffffffu, r);
     };
     for (int j = 0; ok && j < T; ++j) {
-      if (!(ok = wait_warp(s_full, j))) break;
+      if (!(ok = wait_warp(&s_full[w], j))) break;
       tc_fence_after_sync();
       const int k0 = j * 128 + 64 * w;  // first key of this warpgroup's columns
       const bool masked = (k0 + 63 >= p.n_kv) || (CAUSAL && k0 + 63 > q0 + off);
