@@ -23,8 +23,9 @@
 // reference, so the result is exact whatever reference is used.
 //
 // Warp roles (192 threads): warp 0 TMA producer (Q once, then K_j, V_j into a
-// ring of NSLOT 32 KB slots), warp 1 MMA issuer and TMEM owner, warps 2-5 the
-// softmax (one key each) and the epilogue (one output dimension each).
+// ring of NSLOT 32 KB slots -- six, so three K/V tile pairs are in flight from
+// HBM), warp 1 MMA issuer and TMEM owner, warps 2-5 the softmax (one key each)
+// and the epilogue (one output dimension each).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -35,6 +36,9 @@
 #ifndef SDPA_GQA_CHUNK_MAX
 #define SDPA_GQA_CHUNK_MAX 2048
 #endif
+#ifndef SDPA_GQA_NSLOT
+#define SDPA_GQA_NSLOT 6  // 192 KB of ring, one CTA per SM (measured: 6 slots 5.94, 3 slots x 2 CTAs 5.70 TB/s)
+#endif
 
 namespace sdpa {
 
@@ -44,7 +48,7 @@ struct GqaCfg {
   static constexpr int D = 128;
   static constexpr int TILE_BYTES = 128 * D * 2;     // 128 keys x 128 dims, bf16
   static constexpr int BLOCK_BYTES = 128 * 64 * 2;   // one 64-dim swizzle block of a tile
-  static constexpr int NSLOT = 3;                    // ring slots: K_0, V_0, K_1, V_1, ...
+  static constexpr int NSLOT = SDPA_GQA_NSLOT;       // ring slots: K_0, V_0, K_1, V_1, ...
   static constexpr int QP_BLOCK = NQ * 128;          // NQ rows x 64 bf16 (a block of Q or of P^T)
   static constexpr int KV_OFF = 0;
   static constexpr int Q_OFF = NSLOT * TILE_BYTES;
@@ -55,7 +59,7 @@ struct GqaCfg {
   static constexpr int RED_OFF = BAR_OFF + NBAR * 8 + 16;  // after the TMEM slot and abort flag
   static constexpr int SMEM_BYTES = RED_OFF + 4 * NQ * 4 + 1024;
   static constexpr int THREADS = 192;
-  static constexpr int MIN_BLOCKS = (NQ == 16) ? 2 : 1;
+  static constexpr int MIN_BLOCKS = (NQ == 16 && NSLOT <= 3) ? 2 : 1;  // two CTAs per SM fit 3 slots each
   static constexpr uint32_t TMEM_COLS = (3 * NQ <= 64) ? 64u : 128u;
   static constexpr uint32_t COL_O = 2 * NQ;  // S^T buffers at columns [0, NQ) and [NQ, 2 NQ)
 };
