@@ -72,3 +72,30 @@ def test_traffic_is_null_when_kernel_changed(tmp_path, monkeypatch):
     assert bench.profiled_traffic("p.txt", ["k.cuh"]) == 123.0
     src.write_text("kernel v2")
     assert bench.profiled_traffic("p.txt", ["k.cuh"]) is None
+
+
+def test_cost_model_arithmetic():
+    # alpha F + beta M with alpha, beta the reciprocal peaks; the roofline is the larger term
+    import bench
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+    c = bench.cost_model(2e12, 1e10, 0.004, peaks, standard_bytes=3e10)
+    assert abs(c["predicted_ms"] - (2.0 + 2.0)) < 1e-9          # 2e12 / 1e15 s + 1e10 / 5e12 s
+    assert abs(c["roofline_ms"] - 2.0) < 1e-9
+    assert abs(c["measured_over_predicted"] - 1.0) < 1e-9
+    assert abs(c["standard_predicted_ms"] - 8.0) < 1e-9           # 2 ms + 3e10 / 5e12 s
+    assert abs(c["predicted_speedup_vs_standard"] - 2.0) < 1e-9
+
+
+def test_standard_traffic_counts_every_pair():
+    import bench
+    from seeded_inputs import workloads as W
+    w = W.CFG2C  # causal: the standard implementation still forms every (query, key) pair
+    assert bench.standard_bytes(w) == w.bytes() + 4 * 16 * 2048 * 2048 * 12
+
+
+def test_flop_convention():
+    # two matrix products at 2 FLOP per multiply-add; a causal mask halves the count
+    # (the convention of the 2-simplicial article, "model design")
+    from seeded_inputs import workloads as W
+    assert W.CFG2.flops() == 4.0 * 4 * 16 * 2048 * 2048 * 64
+    assert W.CFG2C.flops() == W.CFG2.flops() / 2
