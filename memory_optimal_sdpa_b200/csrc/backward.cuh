@@ -22,12 +22,20 @@
 // Warp roles (384 threads, as the forward kernel): warps 0-7 two elementwise
 // warpgroups (warpgroup w takes columns [64 w, 64 w + 64) of the 128 x 128
 // tile; thread = TMEM lane = the tile's key (dkdv) or query row (dq)), warp 8
-// the TMA producer, warp 9 the MMA issuer and TMEM owner, warps 10-11 idle.
+// the TMA producer, warp 9 the MMA issuer and TMEM owner (at d = 128 only the
+// S / dP one, with warp 10 issuing the gradient products), the rest idle.
 #pragma once
 
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
+
+// At d = 128, two MMA issuers: one for the S / dP products, one for the gradient products
+// (which also releases the ring stages), so neither waits behind the other's instruction
+// stream (measured: d = 128 causal 536 -> 546 TF/s; at d = 64 one issuer is faster, 400 vs 380).
+#ifndef SDPA_BWD_TWO_ISSUERS_MIN_D
+#define SDPA_BWD_TWO_ISSUERS_MIN_D 128
+#endif
 
 namespace sdpa {
 
@@ -56,8 +64,8 @@ struct BwdCfg {
   static constexpr int FIX_OFF = 0;                // the CTA's fixed pair: (K, V) or (Q, dO)
   static constexpr int ST_OFF = 2 * TILE_BYTES;    // streamed stages: (Q, dO, vectors) or (K, V)
   static constexpr int BAR_OFF = ST_OFF + NSTAGE * STAGE_BYTES;
-  // fix_full, full[NSTAGE], empty[NSTAGE], s_full[2], p_full[2], o_full, drain
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 6;
+  // fix_full, full[NSTAGE], empty[NSTAGE], s_full[2], p_full[2], grad_done[2], o_full, drain[2]
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 9;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;
   static constexpr int THREADS = 384;
   static constexpr int EW_REGS = 216;
@@ -69,6 +77,7 @@ struct BwdCfg {
   static constexpr uint32_t COL_A = 256;    // accumulator: dV (dkdv) or dQ (dq)
   static constexpr uint32_t COL_B = 256 + D;  // accumulator: dK (dkdv)
   static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr bool TWO_ISSUERS = D >= SDPA_BWD_TWO_ISSUERS_MIN_D;
 };
 
 // TMEM column of the bf16 pairs holding tile columns [16 kk, 16 kk + 16): warpgroup w packs
@@ -156,8 +165,9 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* empty = full + C::NSTAGE;
   uint64_t* s_full = empty + C::NSTAGE;  // [half]
   uint64_t* p_full = s_full + 2;         // [half] = [warpgroup]
-  uint64_t* o_full = p_full + 2;
-  uint64_t* drain = o_full + 1;
+  uint64_t* grad_done = p_full + 2;      // [half]: the gradient products reading half h completed
+  uint64_t* o_full = grad_done + 2;
+  uint64_t* drain = o_full + 1;          // [issuer]
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -185,8 +195,11 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&s_full[1], 1);
     mbar_init(&p_full[0], 128);
     mbar_init(&p_full[1], 128);
+    mbar_init(&grad_done[0], 1);
+    mbar_init(&grad_done[1], 1);
     mbar_init(o_full, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -235,8 +248,9 @@ __global__ void __launch_bounds__(384, 1)
             mbar_wait_drain(&full[t % C::NSTAGE], (uint32_t)(t / C::NSTAGE) & 1u);
         }
       }
-    } else if (warp == C::MMA_WARP) {
-      // ------------------------------------------------------------ MMA issuer
+    } else if (warp == C::MMA_WARP || (C::TWO_ISSUERS && warp == C::MMA_WARP + 1)) {
+      // ------------------------------------------------------------ MMA issuer(s)
+      const int role = warp - C::MMA_WARP;  // with two issuers: 0 S / dP, 1 gradients
       if (lane == 0 && NT > 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);  // K or V (K-major) x 64 rows of Q or dO
         constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);    // P^T or dS^T (TMEM) x dO or Q (MN-major)
@@ -274,25 +288,45 @@ __global__ void __launch_bounds__(384, 1)
         };
         // Half h of tile t + 1 starts as soon as warpgroup h has finished half h of tile t, so one
         // warpgroup's elementwise pass overlaps the other's and the tensor core's products.
-        bool ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0);
-        if (ok) {
-          issue_sdp(0, 0);
-          issue_sdp(0, 1);
-        }
-        for (int t = 0; ok && t < NT; ++t) {
-          for (int h = 0; ok && h < 2; ++h) {
-            if (!(ok = wait_bar(&p_full[h], t))) break;
-            issue_grad(t, h);
-            if (h == 1) tc_commit(&empty[t % C::NSTAGE]);
-            if (t + 1 < NT) {
-              if (h == 0 && !(ok = wait_bar(&full[(t + 1) % C::NSTAGE], (t + 1) / C::NSTAGE))) break;
-              issue_sdp(t + 1, h);
+        bool ok = true;
+        if (!C::TWO_ISSUERS) {
+          ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0);
+          if (ok) {
+            issue_sdp(0, 0);
+            issue_sdp(0, 1);
+          }
+          for (int t = 0; ok && t < NT; ++t) {
+            for (int h = 0; ok && h < 2; ++h) {
+              if (!(ok = wait_bar(&p_full[h], t))) break;
+              issue_grad(t, h);
+              if (h == 1) tc_commit(&empty[t % C::NSTAGE]);
+              if (t + 1 < NT) {
+                if (h == 0 && !(ok = wait_bar(&full[(t + 1) % C::NSTAGE], (t + 1) / C::NSTAGE))) break;
+                issue_sdp(t + 1, h);
+              }
             }
           }
+          if (ok) tc_commit(o_full);
+        } else if (role == 0) {  // S / dP: half h of tile t once the gradient products of half h of t - 1 are done
+          ok = wait_bar(fix_full, 0);
+          for (int t = 0; ok && t < NT; ++t)
+            for (int h = 0; ok && h < 2; ++h) {
+              if (h == 0 && !(ok = wait_bar(&full[t % C::NSTAGE], t / C::NSTAGE))) break;
+              if (t > 0 && !(ok = wait_bar(&grad_done[h], t - 1))) break;
+              issue_sdp(t, h);
+            }
+        } else {  // gradients: half h of tile t once its elementwise pass is done
+          for (int t = 0; ok && t < NT; ++t)
+            for (int h = 0; ok && h < 2; ++h) {
+              if (!(ok = wait_bar(&p_full[h], t))) break;
+              issue_grad(t, h);
+              tc_commit(&grad_done[h]);
+              if (h == 1) tc_commit(&empty[t % C::NSTAGE]);
+            }
+          if (ok) tc_commit(o_full);
         }
-        if (ok) tc_commit(o_full);
-        tc_commit(drain);
-        mbar_wait_drain(drain, 0);
+        tc_commit(&drain[role]);
+        mbar_wait_drain(&drain[role], 0);
       }
     }
   } else {
@@ -328,11 +362,20 @@ __global__ void __launch_bounds__(384, 1)
         reg_fence(dp);
         uint32_t pp[16], ps[16];
         const int qc = q0 + 32 * h;
+        // this chunk's 32 query vectors, four per 16-byte load (every lane reads the same words)
+        float l2v[32], ddv[32];
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const float4 a = *reinterpret_cast<const float4*>(vL2 + cbase + c);
+          const float4 b = *reinterpret_cast<const float4*>(vD + cbase + c);
+          l2v[c] = a.x, l2v[c + 1] = a.y, l2v[c + 2] = a.z, l2v[c + 3] = a.w;
+          ddv[c] = b.x, ddv[c + 1] = b.y, ddv[c + 2] = b.z, ddv[c + 3] = b.w;
+        }
         if (masked)
-          bwd_elementwise(s, dp, c2, [&](int c) { return vL2[cbase + c]; }, [&](int c) { return vD[cbase + c]; },
+          bwd_elementwise(s, dp, c2, [&](int c) { return l2v[c]; }, [&](int c) { return ddv[c]; },
                           [&](int c) { return key <= qc + c + off; }, pp, ps);
         else
-          bwd_elementwise(s, dp, c2, [&](int c) { return vL2[cbase + c]; }, [&](int c) { return vD[cbase + c]; },
+          bwd_elementwise(s, dp, c2, [&](int c) { return l2v[c]; }, [&](int c) { return ddv[c]; },
                           [&](int) { return true; }, pp, ps);
         tmem_st_32x32b_x16(tmem + C::COL_S + (uint32_t)(64 * w + 16 * h) + lane_base, pp);
         tmem_st_32x32b_x16(tmem + C::COL_DP + (uint32_t)(64 * w + 16 * h) + lane_base, ps);
@@ -402,8 +445,9 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* empty = full + C::NSTAGE;
   uint64_t* s_full = empty + C::NSTAGE;  // [half]
   uint64_t* p_full = s_full + 2;         // [half] = [warpgroup]
-  uint64_t* o_full = p_full + 2;
-  uint64_t* drain = o_full + 1;
+  uint64_t* grad_done = p_full + 2;      // [half]: the gradient products reading half h completed
+  uint64_t* o_full = grad_done + 2;
+  uint64_t* drain = o_full + 1;          // [issuer]
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -430,8 +474,11 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&s_full[1], 1);
     mbar_init(&p_full[0], 128);
     mbar_init(&p_full[1], 128);
+    mbar_init(&grad_done[0], 1);
+    mbar_init(&grad_done[1], 1);
     mbar_init(o_full, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -476,8 +523,9 @@ __global__ void __launch_bounds__(384, 1)
             mbar_wait_drain(&full[j % C::NSTAGE], (uint32_t)(j / C::NSTAGE) & 1u);
         }
       }
-    } else if (warp == C::MMA_WARP) {
-      // ------------------------------------------------------------ MMA issuer
+    } else if (warp == C::MMA_WARP || (C::TWO_ISSUERS && warp == C::MMA_WARP + 1)) {
+      // ------------------------------------------------------------ MMA issuer(s)
+      const int role = warp - C::MMA_WARP;  // with two issuers: 0 S / dP, 1 gradients
       if (lane == 0 && T > 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);  // Q or dO (K-major) x 64 rows of K or V
         constexpr uint32_t idA = idesc_bf16_f32(128, D, false, true);    // dS (TMEM) x K (MN-major)
@@ -507,25 +555,45 @@ __global__ void __launch_bounds__(384, 1)
                    (j > 0 || kk > 0) ? 1u : 0u);
           }
         };
-        bool ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0);
-        if (ok) {
-          issue_sdp(0, 0);
-          issue_sdp(0, 1);
-        }
-        for (int j = 0; ok && j < T; ++j) {
-          for (int h = 0; ok && h < 2; ++h) {
-            if (!(ok = wait_bar(&p_full[h], j))) break;
-            issue_grad(j, h);
-            if (h == 1) tc_commit(&empty[j % C::NSTAGE]);
-            if (j + 1 < T) {
-              if (h == 0 && !(ok = wait_bar(&full[(j + 1) % C::NSTAGE], (j + 1) / C::NSTAGE))) break;
-              issue_sdp(j + 1, h);
+        bool ok = true;
+        if (!C::TWO_ISSUERS) {
+          ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0);
+          if (ok) {
+            issue_sdp(0, 0);
+            issue_sdp(0, 1);
+          }
+          for (int j = 0; ok && j < T; ++j) {
+            for (int h = 0; ok && h < 2; ++h) {
+              if (!(ok = wait_bar(&p_full[h], j))) break;
+              issue_grad(j, h);
+              if (h == 1) tc_commit(&empty[j % C::NSTAGE]);
+              if (j + 1 < T) {
+                if (h == 0 && !(ok = wait_bar(&full[(j + 1) % C::NSTAGE], (j + 1) / C::NSTAGE))) break;
+                issue_sdp(j + 1, h);
+              }
             }
           }
+          if (ok) tc_commit(o_full);
+        } else if (role == 0) {
+          ok = wait_bar(fix_full, 0);
+          for (int j = 0; ok && j < T; ++j)
+            for (int h = 0; ok && h < 2; ++h) {
+              if (h == 0 && !(ok = wait_bar(&full[j % C::NSTAGE], j / C::NSTAGE))) break;
+              if (j > 0 && !(ok = wait_bar(&grad_done[h], j - 1))) break;
+              issue_sdp(j, h);
+            }
+        } else {
+          for (int j = 0; ok && j < T; ++j)
+            for (int h = 0; ok && h < 2; ++h) {
+              if (!(ok = wait_bar(&p_full[h], j))) break;
+              issue_grad(j, h);
+              tc_commit(&grad_done[h]);
+              if (h == 1) tc_commit(&empty[j % C::NSTAGE]);
+            }
+          if (ok) tc_commit(o_full);
         }
-        if (ok) tc_commit(o_full);
-        tc_commit(drain);
-        mbar_wait_drain(drain, 0);
+        tc_commit(&drain[role]);
+        mbar_wait_drain(&drain[role], 0);
       }
     }
   } else {

@@ -136,6 +136,29 @@ def test_prefill_identity_values_give_probabilities(sdpa, cuda_device):
             assert (np.abs(O - P) <= 2 ** -7 * P + 1e-6).all(), "d=%d causal=%d" % (d, causal)
 
 
+@pytest.mark.parametrize("d,causal", [(64, False), (64, True), (128, False), (128, True)])
+def test_prefill_rescale_every_tile(sdpa, cuda_device, d, causal):
+    # Keys grow tile by tile (128-key tiles), so every row's maximum rises by far more than the
+    # lazy threshold (2^8) at each tile: the running sum and O are rescaled at every step.
+    import torch
+    B, H, n = 1, 2, 640
+    g = np.random.default_rng(40 + d)
+    q = np.abs(g.standard_normal((B, H, n, d))).astype(np.float32) * 0.25 + 0.5
+    k = g.standard_normal((B, H, n, d)).astype(np.float32) * 0.05 + (np.arange(n) // 128)[None, None, :, None] * 1.25
+    v = g.standard_normal((B, H, n, d)).astype(np.float32)
+    to = lambda a: torch.from_numpy(a).to(cuda_device).to(torch.bfloat16)
+    tq, tk, tv = to(q), to(k), to(v)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    o, lse = sdpa.fwd(tq, tk, tv, causal=causal, scale=scale)
+    qf, kf, vf = (t.float().cpu().numpy() for t in (tq, tk, tv))  # the bf16 values the kernel saw
+    O_ref, L_ref = oracle.sdpa_rows(qf, kf, vf, scale, causal)
+    check_bf16(o.float().cpu().numpy(), O_ref, lse.cpu().numpy(), L_ref, "rescale d=%d causal=%d" % (d, causal))
+    # the logits really climb past the threshold between tiles
+    s = np.einsum("d,kd->k", qf[0, 0, -1].astype(np.float64), kf[0, 0].astype(np.float64)) * scale / math.log(2)
+    tile_max = s.reshape(-1, 128).max(axis=1)
+    assert (np.diff(tile_max) > 8).all()
+
+
 def test_prefill_lse_optional_and_repeatable(sdpa, cuda_device):
     import torch
     B, H, n, d = 1, 4, 384, 128
