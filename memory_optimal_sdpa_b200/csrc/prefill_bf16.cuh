@@ -58,8 +58,9 @@ struct PrefillCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
-  // q_full, full[NSLOT], empty[NSLOT], s_full[2], s_free[2], p_full[2], pv_done[2], o_full[2], drain[2], turn[8]
-  static constexpr int NBAR = 1 + 2 * NSLOT + 2 * 6 + 8;
+  // q_full, full[NSLOT], empty[NSLOT], s_full[2], s_free[2], p_full[2], pv_done[2], o_full[2], drain[2], turn[8],
+  // q_free, o_free[2]
+  static constexpr int NBAR = 1 + 2 * NSLOT + 2 * 6 + 8 + 3;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;  // + tmem slot, abort flag, align slack
   static constexpr int THREADS = 384;
   static constexpr int SOFTMAX_REGS = 216;
@@ -157,6 +158,14 @@ __device__ __forceinline__ float softmax_exp_row(const uint32_t (&s)[128], float
 
 // MASK: 0 full attention, 1 causal (bottom-right aligned), 2 local window (p.win_left, p.win_right).
 // Modes 0 and 1 fix the bounds at compile time, so their key ranges and masks fold to constants.
+//
+// Persistent: each CTA takes work units (one (batch, head) and two adjacent query tiles) from
+// the unit list, heaviest first, dealt round by round in alternating directions.  TMEM, barriers and descriptor prefetches
+// are set up once; every barrier's phase runs on across units (counters of ring slots, rounds
+// and units per role), and the next unit's Q, K, V loads and first S products proceed while
+// the softmax warpgroups still write the previous unit's output.  Two barriers guard what a
+// unit hands to the next: q_free (both issuers' last S of the unit has run: Q may be
+// replaced) and o_free[x] (the epilogue has read O_x: the next P_x V may overwrite it).
 template <int D, int MASK>
 __global__ void __launch_bounds__(384, 1)
     sdpa_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -177,27 +186,45 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* pv_done = p_full + 2;
   uint64_t* o_full = pv_done + 2;
   uint64_t* drain = o_full + 2;
-  uint64_t* turn = drain + 2;  // [query tile][warp within the warpgroup]
+  uint64_t* turn = drain + 2;      // [query tile][warp within the warpgroup]
+  uint64_t* q_free = turn + 8;     // both issuers' S products of a unit have run
+  uint64_t* o_free = q_free + 1;   // [query tile]: the epilogue has read O_x
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // Work unit: heaviest query-tile pairs (the last rows, under a causal mask) first.
-  const int bh = blockIdx.x % p.bh_count;
-  const int pair = p.n_pairs - 1 - (int)(blockIdx.x / p.bh_count);
-  const int r0a = pair * 256, r0b = pair * 256 + 128;
+  const int n_units = p.bh_count * p.n_pairs;
   const int win_left = MASK == 2 ? p.win_left : -1;
   const int win_right = MASK == 2 ? p.win_right : (MASK == 1 ? 0 : -1);
-  int fa, ta, fb, tb;  // first key tile and tile count of query tiles a and b
-  prefill_kv_range(r0a, p.n_q, p.n_kv, win_left, win_right, &fa, &ta);
-  prefill_kv_range(r0b, p.n_q, p.n_kv, win_left, win_right, &fb, &tb);
-  const int T = ta > tb ? ta : tb;  // softmax rounds
-  // Key tiles loaded: J0 .. J0 + TL - 1, the union of both ranges (ring index 2 (j - J0) for K_j, +1 for V_j).
-  const int J0 = ta == 0 ? fb : (tb == 0 ? fa : (fa < fb ? fa : fb));
-  const int J1 = ta == 0 ? fb + tb - 1 : (tb == 0 ? fa + ta - 1 : (fa + ta > fb + tb ? fa + ta - 1 : fb + tb - 1));
-  const int TL = (ta == 0 && tb == 0) ? 0 : J1 - J0 + 1;
+
+  // The k-th unit of this CTA: units are numbered heaviest first, and successive rounds of
+  // gridDim.x units are dealt in alternating directions, so a CTA that takes a heavy unit in one
+  // round takes a light one in the next (balanced totals under a causal mask).
+  auto unit_of = [&](int k) {
+    const int G = (int)gridDim.x, b = (int)blockIdx.x;
+    return (k & 1) ? (k + 1) * G - 1 - b : k * G + b;
+  };
+  // Geometry of work unit u: heaviest query-tile pairs (the last rows, under a causal mask) first.
+  struct Unit {
+    int bh, r0a, r0b, fa, ta, fb, tb, T, J0, TL;
+  };
+  auto unit_at = [&](int u) {
+    Unit g;
+    g.bh = u % p.bh_count;
+    const int pair = p.n_pairs - 1 - u / p.bh_count;
+    g.r0a = pair * 256;
+    g.r0b = g.r0a + 128;
+    prefill_kv_range(g.r0a, p.n_q, p.n_kv, win_left, win_right, &g.fa, &g.ta);  // first key tile, count
+    prefill_kv_range(g.r0b, p.n_q, p.n_kv, win_left, win_right, &g.fb, &g.tb);
+    g.T = g.ta > g.tb ? g.ta : g.tb;  // softmax rounds
+    // Key tiles loaded: J0 .. J0 + TL - 1, the union of both ranges.
+    const int J1 = g.ta == 0 ? g.fb + g.tb - 1
+                             : (g.tb == 0 ? g.fa + g.ta - 1 : (g.fa + g.ta > g.fb + g.tb ? g.fa + g.ta - 1 : g.fb + g.tb - 1));
+    g.J0 = g.ta == 0 ? g.fb : (g.tb == 0 ? g.fa : (g.fa < g.fb ? g.fa : g.fb));
+    g.TL = (g.ta == 0 && g.tb == 0) ? 0 : J1 - g.J0 + 1;
+    return g;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -211,9 +238,11 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&p_full[x], 128);
       mbar_init(&pv_done[x], 1);
       mbar_init(&o_full[x], 1);
+      mbar_init(&o_free[x], 128);
     }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    mbar_init(q_free, 2);
     for (int w = 0; w < 8; ++w) mbar_init(&turn[w], SDPA_SM_TURN_WARP ? 32 : 128);
     *abort_flag = 0;
     fence_mbar_init();
@@ -233,33 +262,43 @@ __global__ void __launch_bounds__(384, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONTROL_REGS));
     if (warp == C::LOAD_WARP) {
       // ------------------------------------------------------------ TMA producer
-      if (lane == 0 && TL > 0) {
+      if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
-        mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
+        int ring = 0, nu = 0, issued = 0;  // ring base of this unit, units whose Q was loaded, ring indices issued
+        bool ok = true;
+        for (int k = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++k)) {
+          const Unit g = unit_at(u);
+          // Q of this unit replaces the previous unit's once both issuers' S products of it have run.
+          if (nu > 0 && !(ok = mbar_wait_bounded(q_free, (uint32_t)(nu - 1) & 1u, abort_flag, &timed_out))) break;
+          mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
 #pragma unroll
-        for (int x = 0; x < 2; ++x)
+          for (int x = 0; x < 2; ++x)
 #pragma unroll
-          for (int cb = 0; cb < D / 64; ++cb)
-            tma_load_3d(sQ + x * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmQ, q_full, cb * 64, x ? r0b : r0a, bh);
-        int issued = 0;
-        for (int idx = 0; idx < 2 * TL; ++idx) {
-          const int slot = idx % C::NSLOT;
-          const uint32_t ph = (uint32_t)(idx / C::NSLOT) & 1u;
-          if (!mbar_wait_bounded(&empty[slot], ph ^ 1u, abort_flag, &timed_out)) break;
-          mbar_arrive_expect_tx(&full[slot], C::TILE_BYTES);
-          const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
-          uint8_t* dst = sKV + slot * C::TILE_BYTES;
+            for (int cb = 0; cb < D / 64; ++cb)
+              tma_load_3d(sQ + x * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmQ, q_full, cb * 64, x ? g.r0b : g.r0a, g.bh);
+          ++nu;
+          for (int idx = 0; idx < 2 * g.TL; ++idx) {
+            const int gi = ring + idx;
+            const int slot = gi % C::NSLOT;
+            if (!(ok = mbar_wait_bounded(&empty[slot], ((uint32_t)(gi / C::NSLOT) & 1u) ^ 1u, abort_flag, &timed_out)))
+              break;
+            mbar_arrive_expect_tx(&full[slot], C::TILE_BYTES);
+            const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
+            uint8_t* dst = sKV + slot * C::TILE_BYTES;
 #pragma unroll
-          for (int cb = 0; cb < D / 64; ++cb)
-            tma_load_3d(dst + cb * C::BLOCK_BYTES, map, &full[slot], cb * 64, (J0 + (idx >> 1)) * 128, bh);
-          issued = idx + 1;
+            for (int cb = 0; cb < D / 64; ++cb)
+              tma_load_3d(dst + cb * C::BLOCK_BYTES, map, &full[slot], cb * 64, (g.J0 + (idx >> 1)) * 128, g.bh);
+            issued = gi + 1;
+          }
+          if (!ok) break;
+          ring += 2 * g.TL;
         }
         if (*abort_flag) {  // let the copies already in flight land before the CTA exits
-          mbar_wait_drain(q_full, 0);
-          for (int idx = (issued > C::NSLOT ? issued - C::NSLOT : 0); idx < issued; ++idx)
-            mbar_wait_drain(&full[idx % C::NSLOT], (uint32_t)(idx / C::NSLOT) & 1u);
+          if (nu > 0) mbar_wait_drain(q_full, (uint32_t)(nu - 1) & 1u);
+          for (int gi = (issued > C::NSLOT ? issued - C::NSLOT : 0); gi < issued; ++gi)
+            mbar_wait_drain(&full[gi % C::NSLOT], (uint32_t)(gi / C::NSLOT) & 1u);
         }
       }
     } else if (warp == C::MMA_WARP || warp == C::MMA_WARP + 1) {
@@ -268,9 +307,7 @@ __global__ void __launch_bounds__(384, 1)
       // instruction streams (and their barrier waits) proceed in parallel.  Within one
       // stream tcgen05 MMAs execute in issue order, which is what lets P_x alias S_x.
       const int x = warp - C::MMA_WARP;
-      const int tx = x ? tb : ta;
-      const int lead = tx ? (x ? fb : fa) - J0 : TL;  // loaded key tiles before this query tile's first
-      if (lane == 0 && TL > 0) {
+      if (lane == 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
         constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // P (TMEM) x V (MN-major)
         const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
@@ -281,66 +318,84 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t dK = smem_desc_sw128(sKVa, 16, 1024);                     // K-major
         const uint64_t dV = smem_desc_sw128(sKVa, C::BLOCK_BYTES, 1024);         // MN-major
         const uint32_t tS = tmem + C::col_s(x), tP = tmem + C::col_p(x), tO = tmem + C::col_o(x);
-        // r: this query tile's r-th key tile, the (lead + r)-th one loaded
-        auto issue_S = [&](int r) {  // S_x = Q_x K^T
-          const uint64_t b0 = dK + (uint64_t)((((2 * (lead + r)) % C::NSLOT) * C::TILE_BYTES) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = (uint64_t)((((kk >> 2) * C::BLOCK_BYTES) + (kk & 3) * 32) >> 4);
-            mma_ss(tS, dQ + off, b0 + off, idS, kk > 0 ? 1u : 0u);
-          }
-        };
-        auto issue_PV = [&](int r) {  // O_x += P_x V
-          const uint64_t b0 = dV + (uint64_t)((((2 * (lead + r) + 1) % C::NSLOT) * C::TILE_BYTES) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk)
-            mma_ts(tO, tP + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idO, (r > 0 || kk > 0) ? 1u : 0u);
-        };
         auto wait_bar = [&](uint64_t* bar, int phase) {
           const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
           if (r) tc_fence_after_sync();
           return r;
         };
-        auto wait_slot = [&](int idx) { return wait_bar(&full[idx % C::NSLOT], idx / C::NSLOT); };
-
-        bool ok = wait_bar(q_full, 0);
-        // Key tiles only the other query tile uses are released, in order, once they have landed.
-        for (int idx = 0; ok && idx < 2 * lead; ++idx) {
-          if (!(ok = wait_slot(idx))) break;
-          mbar_arrive(&empty[idx % C::NSLOT]);
-        }
-        const int k0 = 2 * lead;  // ring index of this query tile's first K
-        if (ok && tx > 0) {
-          if ((ok = wait_slot(k0))) {
-            issue_S(0);
-            tc_commit(&s_full[x]);
-            tc_commit(&empty[k0 % C::NSLOT]);
+        auto wait_slot = [&](int gi) { return wait_bar(&full[gi % C::NSLOT], gi / C::NSLOT); };
+        // running counts: ring indices of earlier units, units, rounds of tile x, units with rounds
+        int ring = 0, nu = 0, rx = 0, ox = 0;
+        bool ok = true;
+        for (int k = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++k)) {
+          const Unit g = unit_at(u);
+          const int tx = x ? g.tb : g.ta;
+          const int lead = tx ? (x ? g.fb : g.fa) - g.J0 : g.TL;  // loaded key tiles before this tile's first
+          const int k0 = ring + 2 * lead;                         // ring index of this tile's first K
+          // r: this query tile's r-th key tile
+          auto issue_S = [&](int r) {  // S_x = Q_x K^T
+            const uint64_t b0 = dK + (uint64_t)((((k0 + 2 * r) % C::NSLOT) * C::TILE_BYTES) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = (uint64_t)((((kk >> 2) * C::BLOCK_BYTES) + (kk & 3) * 32) >> 4);
+              mma_ss(tS, dQ + off, b0 + off, idS, kk > 0 ? 1u : 0u);
+            }
+          };
+          auto issue_PV = [&](int r) {  // O_x += P_x V
+            const uint64_t b0 = dV + (uint64_t)((((k0 + 2 * r + 1) % C::NSLOT) * C::TILE_BYTES) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 128 / 16; ++kk)
+              mma_ts(tO, tP + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idO, (r > 0 || kk > 0) ? 1u : 0u);
+          };
+          if (!(ok = wait_bar(q_full, nu))) break;
+          // Key tiles only the other query tile uses are released, in order, once they have landed.
+          for (int gi = ring; ok && gi < k0; ++gi) {
+            if (!(ok = wait_slot(gi))) break;
+            mbar_arrive(&empty[gi % C::NSLOT]);
           }
-        }
-        for (int j = 0; ok && j < tx; ++j) {
-          if (C::P_SEPARATE && j + 1 < tx) {
-            // next S as soon as the softmax has read the current one
-            if (!(ok = wait_slot(k0 + 2 * (j + 1)) && wait_bar(&s_free[x], j))) break;
-            issue_S(j + 1);
-            tc_commit(&s_full[x]);
-            tc_commit(&empty[(k0 + 2 * (j + 1)) % C::NSLOT]);
+          if (ok && tx > 0) {
+            // S_x is free once the softmax has read the previous unit's last S_x (with P aliasing
+            // S_x, the previous P_x V was issued first on this stream)
+            if (C::P_SEPARATE && rx > 0) ok = wait_bar(&s_free[x], rx - 1);
+            if (ok && (ok = wait_slot(k0))) {
+              issue_S(0);
+              tc_commit(&s_full[x]);
+              tc_commit(&empty[k0 % C::NSLOT]);
+            }
           }
-          if (!(ok = wait_slot(k0 + 2 * j + 1) && wait_bar(&p_full[x], j))) break;  // V and P_x of tile j
-          issue_PV(j);
-          if (C::P_SEPARATE) tc_commit(&pv_done[x]);
-          if (j == tx - 1) tc_commit(&o_full[x]);
-          tc_commit(&empty[(k0 + 2 * j + 1) % C::NSLOT]);
-          if (!C::P_SEPARATE && j + 1 < tx) {
-            // P_x aliases S_x: the next S_x is issued after P_x V (same stream, in order)
-            if (!(ok = wait_slot(k0 + 2 * (j + 1)))) break;
-            issue_S(j + 1);
-            tc_commit(&s_full[x]);
-            tc_commit(&empty[(k0 + 2 * (j + 1)) % C::NSLOT]);
+          if (ok && tx <= 1) tc_commit(q_free);  // this unit's S products of tile x are all issued
+          for (int j = 0; ok && j < tx; ++j) {
+            if (C::P_SEPARATE && j + 1 < tx) {
+              // next S as soon as the softmax has read the current one
+              if (!(ok = wait_slot(k0 + 2 * (j + 1)) && wait_bar(&s_free[x], rx + j))) break;
+              issue_S(j + 1);
+              tc_commit(&s_full[x]);
+              tc_commit(&empty[(k0 + 2 * (j + 1)) % C::NSLOT]);
+              if (j + 2 == tx) tc_commit(q_free);
+            }
+            if (!(ok = wait_slot(k0 + 2 * j + 1) && wait_bar(&p_full[x], rx + j))) break;  // V and P_x of tile j
+            if (j == 0 && ox > 0 && !(ok = wait_bar(&o_free[x], ox - 1))) break;  // O_x read by the last epilogue
+            issue_PV(j);
+            if (C::P_SEPARATE) tc_commit(&pv_done[x]);
+            if (j == tx - 1) tc_commit(&o_full[x]);
+            tc_commit(&empty[(k0 + 2 * j + 1) % C::NSLOT]);
+            if (!C::P_SEPARATE && j + 1 < tx) {
+              // P_x aliases S_x: the next S_x is issued after P_x V (same stream, in order)
+              if (!(ok = wait_slot(k0 + 2 * (j + 1)))) break;
+              issue_S(j + 1);
+              tc_commit(&s_full[x]);
+              tc_commit(&empty[(k0 + 2 * (j + 1)) % C::NSLOT]);
+              if (j + 2 == tx) tc_commit(q_free);
+            }
           }
-        }
-        for (int idx = k0 + 2 * tx; ok && idx < 2 * TL; ++idx) {
-          if (!(ok = wait_slot(idx))) break;
-          mbar_arrive(&empty[idx % C::NSLOT]);
+          for (int gi = k0 + 2 * tx; ok && gi < ring + 2 * g.TL; ++gi) {
+            if (!(ok = wait_slot(gi))) break;
+            mbar_arrive(&empty[gi % C::NSLOT]);
+          }
+          ring += 2 * g.TL;
+          ++nu;
+          rx += tx;
+          if (tx > 0) ++ox;
         }
         // Every MMA and every commit issued above has landed before TMEM is released
         // and before the CTA's shared memory (which the commits arrive on) goes away.
@@ -353,24 +408,12 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------ softmax + epilogue warpgroups
     const int x = warp >> 2;  // query tile a (0) or b (1)
     const int t = threadIdx.x & 127;
-    const int row = (x ? r0b : r0a) + t;
-    const int tiles = x ? tb : ta;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tS = tmem + C::col_s(x) + lane_base;
     const uint32_t tP = tmem + C::col_p(x) + lane_base;
     const uint32_t tO = tmem + C::col_o(x) + lane_base;
-    // keys this row may see: lo .. lim
-    const int first = x ? fb : fa;
-    int lim = p.n_kv - 1, lo = 0;
-    {
-      const long long pos = (long long)row + p.n_kv - p.n_q;
-      if (win_right >= 0 && pos + win_right < lim) lim = (int)(pos + win_right < -1 ? -1 : pos + win_right);
-      if (win_left >= 0 && pos - win_left > 0) lo = (int)(pos - win_left > p.n_kv ? p.n_kv : pos - win_left);
-    }
     const float c2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
-    float m_u = NEG_INF;  // running max of scale*log2(e)*s
-    float l = 0.f;
     bool ok = true;
     // Waits ahead of warp-collective TMEM instructions: the whole warp proceeds or none of it.
     auto wait_warp = [&](uint64_t* bar, int phase) {
@@ -380,130 +423,155 @@ __global__ void __launch_bounds__(384, 1)
     // The two softmax warpgroups take turns on the exponentials (the MUFU-bound part), so
     // that one's TMEM traffic, row maxima and hand-offs -- and, with P aliasing S, its
     // P V and next S MMAs -- overlap the other's exponentials.  Round j is tile a's turn,
-    // then tile b's; both run T = max(ta, tb) rounds (a round without a tile only passes
-    // the turn).  MUFU units belong to SM sub-partitions, and warp w of each warpgroup
+    // then tile b's; both run T = max(ta, tb) rounds per unit (a round without a tile only
+    // passes the turn).  MUFU units belong to SM sub-partitions, and warp w of each warpgroup
     // runs on sub-partition w, so the turn passes between those two warps alone
-    // (SDPA_SM_TURN_WARP) rather than between whole warpgroups.  my_turn completes phase
-    // j when the other warp hands over; tile b hands tile a its first turn up front.
+    // (SDPA_SM_TURN_WARP) rather than between whole warpgroups.  my_turn completes once per
+    // hand-over; tile b hands tile a its very first turn, and each unit's last hand-over from
+    // b is tile a's first turn of the next unit.
     uint64_t* my_turn = &turn[SDPA_SM_TURN_WARP ? 4 * x + (warp & 3) : 4 * x];
     uint64_t* their_turn = &turn[SDPA_SM_TURN_WARP ? 4 * (x ^ 1) + (warp & 3) : 4 * (x ^ 1)];
     if (SDPA_SM_TURN && x == 1) mbar_arrive(their_turn);
-    for (int j = 0; ok && j < T; ++j) {
-      if (j >= tiles) {  // no key tile left for this query tile: only pass the turn
-        if (SDPA_SM_TURN) {
-          if (!(ok = wait_warp(my_turn, j))) break;
-          mbar_arrive(their_turn);
+    int rx = 0, R = 0, ox = 0;  // rounds of this tile so far, rounds of both, units with rounds
+    for (int k = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++k)) {
+      const Unit g = unit_at(u);
+      const int row = (x ? g.r0b : g.r0a) + t;
+      const int tiles = x ? g.tb : g.ta;
+      // keys this row may see: lo .. lim
+      const int first = x ? g.fb : g.fa;
+      int lim = p.n_kv - 1, lo = 0;
+      {
+        const long long pos = (long long)row + p.n_kv - p.n_q;
+        if (win_right >= 0 && pos + win_right < lim) lim = (int)(pos + win_right < -1 ? -1 : pos + win_right);
+        if (win_left >= 0 && pos - win_left > 0) lo = (int)(pos - win_left > p.n_kv ? p.n_kv : pos - win_left);
+      }
+      float m_u = NEG_INF;  // running max of scale*log2(e)*s
+      float l = 0.f;
+      for (int j = 0; ok && j < g.T; ++j) {
+        if (j >= tiles) {  // no key tile left for this query tile: only pass the turn
+          if (SDPA_SM_TURN) {
+            if (!(ok = wait_warp(my_turn, R + j))) break;
+            mbar_arrive(their_turn);
+          }
+          continue;
         }
-        continue;
-      }
-      uint32_t s[128];
-      if (!(ok = wait_warp(&s_full[x], j))) break;
-      tc_fence_after_sync();
-      tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-      tmem_wait_ld();
-      reg_fence(s);
-      if (C::P_SEPARATE) {  // S_x is in registers: the tensor core may overwrite it with S_x(j+1)
-        tc_fence_before_sync();
-        mbar_arrive(&s_free[x]);
-      }
-      const int kv0 = (first + j) * 128;
-      const bool masked = kv0 + 127 > lim || kv0 < lo;
-      if (masked) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (kv0 + c > lim || kv0 + c < lo) s[c] = __float_as_uint(NEG_INF);
-      }
-      float mx;
-      {  // eight independent chains of 3-input maxima over s[0..127]: 16 + 7 x 16 scores
-        float m[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) m[k] = fmaxf(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1]));
-#pragma unroll
-        for (int c = 16; c < 128; c += 16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) m[k] = max3f(m[k], __uint_as_float(s[c + 2 * k]), __uint_as_float(s[c + 2 * k + 1]));
-        mx = max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
-      }
-      const float m_new = fmaxf(m_u, mx * c2);
-      const bool need = m_new > m_u + 8.0f;
-      bool pv_waited = false;  // P_x V of the previous tile known complete (P_x and O_x free)
-      if (__any_sync(0xffffffffu, need)) {
-        float alpha = 1.f;
-        if (m_new > m_u) {
-          alpha = ex2_approx(m_u - m_new);  // 0 when m_u = -inf
-          m_u = m_new;
-          l *= alpha;
+        uint32_t s[128];
+        if (!(ok = wait_warp(&s_full[x], rx + j))) break;
+        tc_fence_after_sync();
+        tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+        tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+        tmem_wait_ld();
+        reg_fence(s);
+        if (C::P_SEPARATE) {  // S_x is in registers: the tensor core may overwrite it with the next S_x
+          tc_fence_before_sync();
+          mbar_arrive(&s_free[x]);
         }
-        if (j > 0) {  // O_x holds P V of earlier tiles
-          if (C::P_SEPARATE) {
-            if (!(ok = wait_warp(&pv_done[x], j - 1))) break;
-            tc_fence_after_sync();
-            pv_waited = true;
-          }  // (aliased P: S_x(j) was issued after P_x V of tile j-1, so that is complete)
+        const int kv0 = (first + j) * 128;
+        const bool masked = kv0 + 127 > lim || kv0 < lo;
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (kv0 + c > lim || kv0 + c < lo) s[c] = __float_as_uint(NEG_INF);
+        }
+        float mx;
+        {  // eight independent chains of 3-input maxima over s[0..127]: 16 + 7 x 16 scores
+          float m[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m[k] = fmaxf(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1]));
+#pragma unroll
+          for (int c = 16; c < 128; c += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              m[k] = max3f(m[k], __uint_as_float(s[c + 2 * k]), __uint_as_float(s[c + 2 * k + 1]));
+          mx = max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+        }
+        const float m_new = fmaxf(m_u, mx * c2);
+        const bool need = m_new > m_u + 8.0f;
+        bool pv_waited = false;  // P_x V of the previous round known complete (P_x and O_x free)
+        if (__any_sync(0xffffffffu, need)) {
+          float alpha = 1.f;
+          if (m_new > m_u) {
+            alpha = ex2_approx(m_u - m_new);  // 0 when m_u = -inf
+            m_u = m_new;
+            l *= alpha;
+          }
+          if (j > 0) {  // O_x holds P V of earlier tiles of this unit
+            if (C::P_SEPARATE) {
+              if (!(ok = wait_warp(&pv_done[x], rx + j - 1))) break;
+              tc_fence_after_sync();
+              pv_waited = true;
+            }  // (aliased P: S_x(j) was issued after P_x V of tile j-1, so that is complete)
 #pragma unroll 1
-          for (int cb = 0; cb < D; cb += 32) {
-            uint32_t o[32];
+            for (int cb = 0; cb < D; cb += 32) {
+              uint32_t o[32];
+              tmem_ld_32x32b_x32(tO + cb, o);
+              tmem_wait_ld();
+              reg_fence(o);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st_32x32b_x32(tO + cb, o);
+            }
+          }
+        }
+        if (SDPA_SM_TURN && !(ok = wait_warp(my_turn, R + j))) break;  // this warp's turn on the exponentials
+        const float m_use = (m_u == NEG_INF) ? 0.f : m_u;
+        uint32_t pk[64];
+        l += masked ? softmax_exp_row<false>(s, c2, m_use, pk) : softmax_exp_row<true>(s, c2, m_use, pk);
+        if (SDPA_SM_TURN) mbar_arrive(their_turn);  // hand the exponentials over
+        if (C::P_SEPARATE && rx + j > 0 && !pv_waited) {  // the last P_x V (this unit's or the previous one's) reads P_x
+          if (!(ok = wait_warp(&pv_done[x], rx + j - 1))) break;
+          tc_fence_after_sync();
+        }
+        tmem_st_32x32b_x32(tP + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st_32x32b_x32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        tmem_wait_st();
+        tc_fence_before_sync();
+#ifdef SDPA_FAULT_DROP_ARRIVE
+        // Test builds only: tile b never reports its first P, so its MMA issuer's wait runs out.
+        if (!(x == 1 && j == 0))
+#endif
+          mbar_arrive(&p_full[x]);
+      }
+      // ---------------------------------------------------------------- epilogue
+      if (ok && tiles > 0) ok = wait_warp(&o_full[x], ox);
+      if (ok) {
+        tc_fence_after_sync();
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const bool store = row < p.n_q;
+        uint4* orow = reinterpret_cast<uint4*>(p.O + ((size_t)g.bh * p.n_q + (store ? row : 0)) * D);
+#pragma unroll 1
+        for (int cb = 0; cb < D; cb += 32) {
+          uint32_t o[32];
+          if (tiles > 0) {
             tmem_ld_32x32b_x32(tO + cb, o);
             tmem_wait_ld();
             reg_fence(o);
+          } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st_32x32b_x32(tO + cb, o);
+            for (int i = 0; i < 32; ++i) o[i] = 0u;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          if (store) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              orow[cb / 8 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
           }
         }
-      }
-      if (SDPA_SM_TURN && !(ok = wait_warp(my_turn, j))) break;  // this warp's turn on the exponentials
-      const float m_use = (m_u == NEG_INF) ? 0.f : m_u;
-      uint32_t pk[64];
-      l += masked ? softmax_exp_row<false>(s, c2, m_use, pk) : softmax_exp_row<true>(s, c2, m_use, pk);
-      if (SDPA_SM_TURN) mbar_arrive(their_turn);  // hand the exponentials over
-      if (C::P_SEPARATE && j > 0 && !pv_waited) {  // P_x V of tile j-1 still reads P_x
-        if (!(ok = wait_warp(&pv_done[x], j - 1))) break;
-        tc_fence_after_sync();
-      }
-      tmem_st_32x32b_x32(tP + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st_32x32b_x32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-      tmem_wait_st();
-      tc_fence_before_sync();
-#ifdef SDPA_FAULT_DROP_ARRIVE
-      // Test builds only: tile b never reports its first P, so its MMA issuer's wait runs out.
-      if (!(x == 1 && j == 0))
-#endif
-        mbar_arrive(&p_full[x]);
-    }
-    // ---------------------------------------------------------------- epilogue
-    if (ok && tiles > 0) ok = wait_warp(&o_full[x], 0);
-    if (ok) {
-      tc_fence_after_sync();
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const bool store = row < p.n_q;
-      uint4* orow = reinterpret_cast<uint4*>(p.O + ((size_t)bh * p.n_q + (store ? row : 0)) * D);
-#pragma unroll 1
-      for (int cb = 0; cb < D; cb += 32) {
-        uint32_t o[32];
-        if (tiles > 0) {
-          tmem_ld_32x32b_x32(tO + cb, o);
-          tmem_wait_ld();
-          reg_fence(o);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        if (tiles > 0) {  // O_x has been read: the next unit's first P_x V may overwrite it
+          tc_fence_before_sync();
+          mbar_arrive(&o_free[x]);
         }
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-        if (store) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            orow[cb / 8 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-        }
+        if (store && p.LSE)
+          p.LSE[(size_t)g.bh * p.n_q + row] = (l > 0.f) ? m_u * 0.69314718055994531f + logf(l) : NEG_INF;
       }
-      if (store && p.LSE)
-        p.LSE[(size_t)bh * p.n_q + row] = (l > 0.f) ? m_u * 0.69314718055994531f + logf(l) : NEG_INF;
+      rx += tiles;
+      R += g.T;
+      if (tiles > 0) ++ox;
     }
   }
 

@@ -70,6 +70,15 @@ bool make_map(CUtensorMap* map, const void* ptr, int d, int n, int bh, int box_r
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Multiprocessors of the current device (the persistent prefill grid).
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0)
+    return 148;
+  return n;
+}
 bool aligned4(const void* p) { return ((uintptr_t)p & 3u) == 0; }
 
 // The current device must be an sm_100 part (B200 class).
@@ -108,7 +117,9 @@ int launch_prefill(const void* Q, const void* K, const void* V, void* O, float* 
   p.scale_log2 = scale * 1.4426950408889634f;
   p.win_left = win_left;
   p.win_right = win_right;
-  const long long grid = (long long)bh * p.n_pairs;
+  // persistent: one CTA per SM (at most one per work unit), each striding over the units
+  long long grid = (long long)bh * p.n_pairs;
+  if (grid > sm_count()) grid = sm_count();
   kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess && debug_on()) {
