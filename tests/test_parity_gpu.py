@@ -159,6 +159,26 @@ def test_prefill_rescale_every_tile(sdpa, cuda_device, d, causal):
     assert (np.diff(tile_max) > 8).all()
 
 
+@pytest.mark.parametrize("d,mode", [(64, "full"), (64, "causal"), (128, "full"), (128, "causal"), (128, "window")])
+def test_prefill_many_units_per_cta(sdpa, cuda_device, d, mode):
+    # 96 (batch, head) slices of 384 rows = 192 work units of two query tiles (the second one
+    # ragged): more units than SMs, so CTAs run several units back to back and every hand-over
+    # between units (Q reload, O read-out, barrier phases) is checked on every row.
+    import torch
+    B, H, n = 8, 12, 384
+    q, k, v = (si.fill_host((B, H, n, d), 60 + d, s_) for s_ in (0, 1, 2))
+    scale = float(np.float32(1 / math.sqrt(d)))
+    tq, tk, tv = (W.to_torch(x, cuda_device) for x in (q, k, v))
+    if mode == "window":
+        o, lse = sdpa.fwd_window(tq, tk, tv, 100, 0, scale=scale)
+        O_ref, L_ref = oracle.sdpa_rows_window(*(si.bf16_bits_to_f32(x) for x in (q, k, v)), scale, 100, 0)
+    else:
+        o, lse = sdpa.fwd(tq, tk, tv, causal=(mode == "causal"), scale=scale)
+        O_ref, L_ref = oracle.sdpa_rows(*(si.bf16_bits_to_f32(x) for x in (q, k, v)), scale, mode == "causal")
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    check_bf16(o.float().cpu().numpy(), O_ref, lse.cpu().numpy(), L_ref, "many units d=%d %s" % (d, mode))
+
+
 def test_prefill_lse_optional_and_repeatable(sdpa, cuda_device):
     import torch
     B, H, n, d = 1, 4, 384, 128
@@ -328,6 +348,23 @@ def test_decode_gqa_small_every_pair(sdpa, cuda_device, B, H_q, H_kv, n_cap, d, 
     check_bf16(o.float().cpu().numpy().reshape(B * H_q, d), O_ref, lse.cpu().numpy().reshape(-1), L_ref,
                "gqa %s" % ((B, H_q, H_kv, n_cap, d, tuple(lens)),))
     assert torch.isnan(o_flat[o.numel():]).all() and torch.isnan(l_flat[lse.numel():]).all()
+
+
+def test_decode_gqa_many_units_per_cta(sdpa, cuda_device):
+    # 48 x 16 key/value heads, one split each of one or two 128-key tiles: 768 units for the
+    # persistent CTAs (several per CTA), lengths from 1 to the full cache, every pair checked
+    import torch
+    B, H_q, H_kv, n_cap, d = 48, 64, 16, 256, 128
+    lens = si.kv_lengths(B, 1, n_cap, 77)
+    lens[:3] = (1, 128, 129)
+    q, k, v = _gqa_inputs(B, H_q, H_kv, n_cap, d, lens, 77)
+    tq, tk, tv = (W.to_torch(x, cuda_device) for x in (q, k, v))
+    tl = torch.from_numpy(lens).to(cuda_device)
+    o, lse = sdpa.decode_gqa(tq, tk, tv, tl, scale=0.09)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O_ref, L_ref = oracle.decode_gqa(*(si.bf16_bits_to_f32(x) for x in (q, k, v)), lens, 0.09)
+    check_bf16(o.float().cpu().numpy().reshape(B * H_q, d), O_ref, lse.cpu().numpy().reshape(-1), L_ref,
+               "gqa many units")
 
 
 def test_decode_gqa_group_of_one_is_decode(sdpa, cuda_device):
