@@ -68,8 +68,8 @@ struct BwdCfg {
   static constexpr int NBAR = 1 + 2 * NSTAGE + 9;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;
   static constexpr int THREADS = 384;
-  static constexpr int EW_REGS = 216;
-  static constexpr int CONTROL_REGS = 72;
+  static constexpr int EW_REGS = 192;  // 192 x 256 + 120 x 128 = 168 x 384: no spills in the control warps
+  static constexpr int CONTROL_REGS = 120;
   static constexpr int LOAD_WARP = 8;
   static constexpr int MMA_WARP = 9;
   static constexpr uint32_t COL_S = 0;      // S or S^T, fp32; then P^T (bf16 pairs) over its first columns
