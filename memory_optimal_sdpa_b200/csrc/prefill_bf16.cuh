@@ -34,18 +34,18 @@
 // The online softmax keeps, per row, the running maximum m (in log2 units of
 // the scaled logits) and sum l; O and l are rescaled only when m grows by more
 // than 8 (a factor 256): O and l always share the same reference maximum, so
-// O/l is exact whatever reference is used, and fp32 cannot overflow.  On tiles
-// without masked entries one column pair in SDPA_EXP2_POLY_EVERY takes its
-// exponentials on the FMA pipe (sm100::exp2_poly2) instead of the MUFU unit,
-// which is the softmax's bottleneck.
+// O/l is exact whatever reference is used, and fp32 cannot overflow.  At d = 64,
+// on tiles without masked entries, one column pair in eight takes its
+// exponentials on the FMA pipe (sm100::exp2_poly2) instead of the MUFU unit
+// (measured: cfg2 537 -> 551 TF/s; at d = 128 it does not pay).
 #pragma once
 
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
 
-#ifndef SDPA_EXP2_POLY_EVERY
-#define SDPA_EXP2_POLY_EVERY 0
+#ifndef SDPA_EXP2_POLY_EVERY_D64
+#define SDPA_EXP2_POLY_EVERY_D64 8  // every 8th column pair of an unmasked tile on the FMA pipe at d = 64
 #endif
 
 namespace sdpa {
@@ -69,6 +69,7 @@ struct PrefillCfg {
   static constexpr int MMA_WARP = 9;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr bool P_SEPARATE = (D == 64);
+  static constexpr int POLY_EVERY = (D == 64) ? SDPA_EXP2_POLY_EVERY_D64 : 0;  // FMA-pipe exponentials
   __host__ __device__ static constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
   __host__ __device__ static constexpr uint32_t col_p(int x) { return P_SEPARATE ? 256u + (uint32_t)x * 64u : col_s(x); }
   __host__ __device__ static constexpr uint32_t col_o(int x) {
@@ -129,8 +130,8 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
 }
 
 // Exponentials of one 128-score row: p = 2^(s*c2 - m), bf16 pairs into pk, returns sum p.
-// POLY: every SDPA_EXP2_POLY_EVERY-th pair on the FMA pipe (finite scores only).
-template <bool POLY>
+// EVERY > 0: every EVERY-th pair on the FMA pipe (finite scores only).
+template <int EVERY>
 __device__ __forceinline__ float softmax_exp_row(const uint32_t (&s)[128], float c2, float m_use, uint32_t (&pk)[64]) {
   using namespace sm100;
   const float2 cc = make_float2(c2, c2), nm = make_float2(-m_use, -m_use);
@@ -139,8 +140,7 @@ __device__ __forceinline__ float softmax_exp_row(const uint32_t (&s)[128], float
   for (int i = 0; i < 64; ++i) {
     const float2 xv = ffma2(make_float2(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), cc, nm);
     float2 e;
-    if (POLY && SDPA_EXP2_POLY_EVERY > 0 && (i % (SDPA_EXP2_POLY_EVERY > 0 ? SDPA_EXP2_POLY_EVERY : 1)) ==
-                                                 SDPA_EXP2_POLY_EVERY - 1) {
+    if (EVERY > 0 && (i % (EVERY > 0 ? EVERY : 1)) == EVERY - 1) {
       e = exp2_poly2(xv);
     } else {
       e.x = ex2_approx(xv.x);
@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(384, 1)
         if (SDPA_SM_TURN && !(ok = wait_warp(my_turn, R + j))) break;  // this warp's turn on the exponentials
         const float m_use = (m_u == NEG_INF) ? 0.f : m_u;
         uint32_t pk[64];
-        l += masked ? softmax_exp_row<false>(s, c2, m_use, pk) : softmax_exp_row<true>(s, c2, m_use, pk);
+        l += masked ? softmax_exp_row<0>(s, c2, m_use, pk) : softmax_exp_row<C::POLY_EVERY>(s, c2, m_use, pk);
         if (SDPA_SM_TURN) mbar_arrive(their_turn);  // hand the exponentials over
         if (C::P_SEPARATE && rx + j > 0 && !pv_waited) {  // the last P_x V (this unit's or the previous one's) reads P_x
           if (!(ok = wait_warp(&pv_done[x], rx + j - 1))) break;
