@@ -242,6 +242,27 @@ def test_cfg4_long_sampled(sdpa, cuda_device):
     _sampled_prefill(sdpa, cuda_device, W.CFG4, 256)
 
 
+@pytest.mark.parametrize("d,causal", [(64, True), (128, False)])
+def test_prefill_long_sequence_sampled(sdpa, cuda_device, d, causal):
+    # n = 131072: four times cfg4's sequence (8.8 TFLOP of tile work at d = 128), one head; the
+    # first, last and seeded interior rows against the oracle
+    import torch
+    n = 131072
+    w = W.Prefill("long%d" % d, 1, 1, n, n, d, causal, "bf16", 1 / d ** 0.5)
+    host = W.prefill_host(w)
+    tq, tk, tv = (W.to_torch(host[x], cuda_device) for x in ("q", "k", "v"))
+    o, lse = sdpa.fwd(tq, tk, tv, causal=causal, scale=w.scale_f32)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    rows = si.sample_rows(n, 48, 0, salt=d)
+    O = o[0, 0, rows].float().cpu().numpy()
+    L = lse[0, 0, rows].cpu().numpy()
+    del tq, tk, tv, o, lse
+    torch.cuda.empty_cache()
+    O_ref, L_ref = oracle.sdpa_rows(*(W.as_f32(host[x])[0, 0] for x in ("q", "k", "v")), w.scale_f32, causal,
+                                    rows=rows)
+    check_bf16(O, O_ref, L, L_ref, "n=%d d=%d causal=%d" % (n, d, causal))
+
+
 # ------------------------------------------------------------------------------------- local windows (bf16)
 WINDOW_CASES = [
     # (B, H, n_q, n_kv, d, left, right)
@@ -365,6 +386,34 @@ def test_decode_gqa_many_units_per_cta(sdpa, cuda_device):
     O_ref, L_ref = oracle.decode_gqa(*(si.bf16_bits_to_f32(x) for x in (q, k, v)), lens, 0.09)
     check_bf16(o.float().cpu().numpy().reshape(B * H_q, d), O_ref, lse.cpu().numpy().reshape(-1), L_ref,
                "gqa many units")
+
+
+def test_decode_gqa_long_cache(sdpa, cuda_device):
+    # a 65536-row cache (four times cfg5g's), groups of 8: one sequence at full length, one short
+    import torch
+    B, H_q, H_kv, n_cap, d = 2, 16, 2, 65536, 128
+    lens = np.array([n_cap, 3000], np.int32)
+    tl = torch.from_numpy(lens).to(cuda_device)
+    tk = torch.empty((B, H_kv, n_cap, d), dtype=torch.bfloat16, device=cuda_device)
+    tv = torch.empty_like(tk)
+    si.fill_device_cache(tk, tl, 5, si.STREAM_K)
+    si.fill_device_cache(tv, tl, 5, si.STREAM_V)
+    q = si.fill_host((B, H_q, d), 5, si.STREAM_Q)
+    o, lse = sdpa.decode_gqa(W.to_torch(q, cuda_device), tk, tv, tl, scale=0.0884)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O = o.float().cpu().numpy()
+    L = lse.cpu().numpy()
+    G = H_q // H_kv
+    for b in range(B):
+        for kvh in range(H_kv):
+            n = int(lens[b])
+            start = ((b * H_kv + kvh) * n_cap) * d
+            kf = si.bf16_bits_to_f32(si.fill_host((1, 1, n, d), 5, si.STREAM_K, start=start))
+            vf = si.bf16_bits_to_f32(si.fill_host((1, 1, n, d), 5, si.STREAM_V, start=start))
+            hs = slice(kvh * G, kvh * G + G)
+            O_ref, L_ref = oracle.decode_gqa(si.bf16_bits_to_f32(q[b:b + 1, hs]), kf, vf, np.array([n], np.int32),
+                                             0.0884)
+            check_bf16(O[b, hs], O_ref, L[b, hs], L_ref, "long cache b=%d kv head %d" % (b, kvh))
 
 
 def test_decode_gqa_group_of_one_is_decode(sdpa, cuda_device):
