@@ -166,7 +166,8 @@ SDPA_API int sdpa_decode_noalloc(const void* Q, const void* K, const void* V, co
 
 /*
  * sdpa_bwd_workspace_size -- bytes of device workspace sdpa_bwd needs:
- * 2 * batch * heads * round_up(n_q, 128) floats.  0 for a degenerate shape.
+ * 2 * batch * heads * round_up(n_q, 128) floats (the per-row vectors D and LSE log2(e)).
+ * 0 for a degenerate shape.
  */
 SDPA_API size_t sdpa_bwd_workspace_size(int batch, int heads, int n_q);
 
@@ -181,7 +182,8 @@ SDPA_API size_t sdpa_bwd_workspace_size(int batch, int heads, int n_q);
  * Q, O, dO, dQ [batch, heads, n_q, d]; K, V, dK, dV [batch, heads, n_kv, d]; all
  * __nv_bfloat16, contiguous, 16-byte aligned.  LSE [batch, heads, n_q] float as sdpa_fwd wrote
  * it (required).  d_k == d_v in {64, 128}; scale > 0 and causal as in the forward call.
- * workspace: caller-owned device memory of sdpa_bwd_workspace_size bytes (scratch).
+ * workspace: caller-owned device memory of sdpa_bwd_workspace_size bytes (scratch, rewritten
+ * by every call: calls that may run at the same time need separate workspaces).
  * Rows whose window held no key (causal, n_q > n_kv) contribute nothing and get dQ = 0.
  * Errors as sdpa_fwd, plus SDPA_ERR_WORKSPACE.
  */

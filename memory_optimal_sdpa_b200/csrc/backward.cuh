@@ -15,7 +15,8 @@
 //         P^T and dS^T (bf16, written back over S^T and dP^T), then dV += P^T dO and
 //         dK += dS^T Q with the TMEM operand form; dV and dK stay in TMEM to the end
 //   dq    one CTA per 128-row query tile, streaming key tiles: S, dP, dS as above,
-//         then dQ += dS K
+//         then dQ += dS K; launched as a programmatic dependent of dkdv (which it does not
+//         read), so its CTAs fill the SMs dkdv's tail leaves
 // Each gradient is written once, so global traffic is O(n d) per kernel and no
 // atomics are needed; the price is computing S and dP in both kernels.
 //
@@ -79,6 +80,15 @@ struct BwdCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr bool TWO_ISSUERS = D >= SDPA_BWD_TWO_ISSUERS_MIN_D;
 };
+
+// Programmatic dependent launch.  launch_dependents: the next kernel on the stream, if launched
+// with programmatic stream serialization, may start once every CTA of this grid has executed it
+// (or exited).  wait: block until the grids this one depends on have completed and their memory
+// operations are visible (returns at once when there are none).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // TMEM column of the bf16 pairs holding tile columns [16 kk, 16 kk + 16): warpgroup w packs
 // its 64 columns into [64 w, 64 w + 32) of the fp32 region it read them from.
@@ -155,6 +165,9 @@ __global__ void __launch_bounds__(384, 1)
                          const BwdParams p) {
   using C = BwdCfg<D>;
   using namespace sm100;
+  // The dQ kernel after this one on the stream reads nothing it writes: once every CTA of this
+  // grid has started, its CTAs may take the SMs this grid's tail leaves.
+  griddep_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sFix = smem + C::FIX_OFF;  // K, V
@@ -258,7 +271,9 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t dK = smem_desc_sw128(fix, 16, 1024);
         const uint64_t dV = smem_desc_sw128(fix + C::TILE_BYTES, 16, 1024);
         auto wait_bar = [&](uint64_t* bar, int phase) {
-          return mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
+          const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
+          if (r) tc_fence_after_sync();  // the elementwise warps' TMEM stores precede the products
+          return r;
         };
         // Query tile t is taken in two halves of 64 rows; half h's S^T and dP^T go to columns
         // [64 h, 64 h + 64) of their regions, where warpgroup h reads them.
@@ -533,7 +548,9 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t dQk = smem_desc_sw128(fix, 16, 1024);
         const uint64_t dOk = smem_desc_sw128(fix + C::TILE_BYTES, 16, 1024);
         auto wait_bar = [&](uint64_t* bar, int phase) {
-          return mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
+          const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
+          if (r) tc_fence_after_sync();  // the elementwise warps' TMEM stores precede the products
+          return r;
         };
         auto issue_sdp = [&](int j, int h) {  // S_h = Q K_h^T, dP_h = dO V_h^T (64 keys)
           const uint32_t sk = st0 + (j % C::NSTAGE) * C::STAGE_BYTES + h * 8192;
@@ -605,8 +622,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const float c2 = p.scale_log2;
     const size_t vi = (size_t)bh * p.n_q_pad + q;  // inside the padded vectors for every lane
-    const float l2 = p.L2[vi];
-    const float dd = p.Dvec[vi];
+    // written by the pre kernel: read through L2 (this grid may start before dkdv has finished)
+    const float l2 = __ldcg(p.L2 + vi);
+    const float dd = __ldcg(p.Dvec + vi);
     bool ok = true;
     auto wait_warp = [&](uint64_t* bar, int phase) {
       const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
@@ -671,6 +689,9 @@ __global__ void __launch_bounds__(384, 1)
     }
   }
 
+  // dkdv, before this kernel on the stream, may still be finishing (it let this one start early):
+  // the stream must see both done when this grid completes.
+  if (threadIdx.x == 0) griddep_wait();
   if (timed_out) record_error(6 /* SDPA_ERR_DEVICE_TIMEOUT */);
   tc_fence_before_sync();
   __syncthreads();

@@ -491,8 +491,21 @@ int launch_bwd(const void* Q, const void* K, const void* V, const sdpa::BwdParam
   sdpa::sdpa_bwd_pre_kernel<D><<<dim3((unsigned)(p.n_q_pad / 128), (unsigned)p.bh_count), 128, 0, stream>>>(p);
   const long long n_kt = (p.n_kv + 127) / 128, n_qt = (p.n_q + 127) / 128;
   kdkdv<<<(unsigned)(p.bh_count * n_kt), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
-  kdq<<<(unsigned)(p.bh_count * n_qt), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
-  const cudaError_t e = cudaGetLastError();
+  // dq reads only what the pre kernel wrote (complete before dkdv started), so it is launched as a
+  // programmatic dependent: its CTAs start on the SMs dkdv's last wave leaves, and it waits for
+  // dkdv itself before it completes.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.bh_count * n_qt));
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, kdq, mq, mk, mv, mdo, p);
   return e == cudaSuccess ? SDPA_OK : cuda_fail("backward launch", e);
 }
 }  // namespace

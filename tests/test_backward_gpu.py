@@ -149,3 +149,31 @@ def test_bwd_cfg2_full_size_four_slices(sdpa, cuda_device, causal):
 def test_bwd_d128_causal_medium(sdpa, cuda_device):
     w = W.Prefill("bwd_d128", 1, 8, 2048, 2048, 128, True, "bf16", 1 / 128 ** 0.5, v=W.Dist(si.UNIFORM, -1.0, 1.0))
     _sampled_slices(sdpa, cuda_device, w, [(0, 0), (0, 3), (0, 7)], True)
+
+
+MANY_UNITS = [
+    # (B, H, n_q, n_kv, d, causal): more 128-row units than SMs, so each persistent CTA walks
+    # several units (ragged tails; the last case has query tiles that see no key)
+    (2, 80, 333, 333, 64, True), (1, 160, 200, 300, 128, False), (2, 96, 300, 200, 64, False),
+    (2, 80, 333, 100, 64, True), (1, 96, 640, 512, 128, True),
+]
+
+
+@pytest.mark.parametrize("B,H,n_q,n_kv,d,causal", MANY_UNITS)
+def test_bwd_many_units_per_cta(sdpa, cuda_device, B, H, n_q, n_kv, d, causal):
+    seed = 900 + n_q + n_kv + d + int(causal)
+    q = si.fill_host((B, H, n_q, d), seed, 0)
+    k = si.fill_host((B, H, n_kv, d), seed, 1)
+    v = si.fill_host((B, H, n_kv, d), seed, 2)
+    do = si.fill_host((B, H, n_q, d), seed, si.STREAM_DO)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    dq, dk, dv = run_bwd(sdpa, cuda_device, q, k, v, do, causal, scale)
+    # every element of every 7th slice, so each CTA position in the dealing is sampled
+    for i in range(0, B * H, 7):
+        b, h = divmod(i, H)
+        qf, kf, vf, dof = (si.bf16_bits_to_f32(x[b, h]) for x in (q, k, v, do))
+        dQ, dK, dV = oracle.sdpa_backward(qf, kf, vf, dof, scale, causal)
+        check_slice(dq[b, h], dk[b, h], dv[b, h], dQ, dK, dV, qf, kf, vf, dof, scale, causal,
+                    "%s b=%d h=%d" % ((B, H, n_q, n_kv, d, causal), b, h))
+    if causal and n_q > n_kv:
+        assert (dq[:, :, :n_q - n_kv] == 0).all()
