@@ -177,3 +177,27 @@ def test_bwd_many_units_per_cta(sdpa, cuda_device, B, H, n_q, n_kv, d, causal):
                     "%s b=%d h=%d" % ((B, H, n_q, n_kv, d, causal), b, h))
     if causal and n_q > n_kv:
         assert (dq[:, :, :n_q - n_kv] == 0).all()
+
+
+def test_bwd_complete_for_work_queued_behind_it(sdpa, cuda_device):
+    # dq runs as a programmatic dependent of dkdv (it may start on SMs dkdv's last wave leaves), so
+    # the stream must still order later work after all three gradients: copies queued right behind
+    # sdpa_bwd, with no synchronisation in between, must equal the gradients read after a sync.
+    import torch
+    w = W.CFG2
+    host = W.prefill_host(w)
+    q, k, v = (W.to_torch(host[n], cuda_device) for n in ("q", "k", "v"))
+    do = W.to_torch(si.fill_host((w.batch, w.heads, w.n_q, w.d), w.seed, si.STREAM_DO), cuda_device)
+    for causal in (False, True):
+        o, lse = sdpa.fwd(q, k, v, causal=causal, scale=w.scale_f32)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        for _ in range(3):
+            for g in (dq, dk, dv):
+                g.zero_()
+            sdpa.bwd(q, k, v, o, do, lse, causal=causal, scale=w.scale_f32, dq=dq, dk=dk, dv=dv)
+            copies = [g.clone() for g in (dq, dk, dv)]  # same stream, queued behind the backward
+            torch.cuda.synchronize()
+            for name, c, g in zip(("dQ", "dK", "dV"), copies, (dq, dk, dv)):
+                assert torch.equal(c, g), "%s read behind sdpa_bwd differs (causal=%s)" % (name, causal)
+            assert dv.abs().sum().item() > 0
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
