@@ -66,9 +66,10 @@ typedef enum {
  * Q, K, V, O: __nv_bfloat16, layout above.  LSE: float or NULL.
  * d_k == d_v, and both in {64, 128} (else SDPA_ERR_UNSUPPORTED).
  * n_q >= 0, n_kv >= 1.  batch*heads*max(n_q, n_kv) < 2^31.
- * causal: 0 or 1.  scale: finite (else SDPA_ERR_INVALID_ARG) and > 0 (else
- * SDPA_ERR_UNSUPPORTED; the online softmax tracks the row maximum of the raw
- * scores, which is the maximum of the scaled ones only for a positive scale).
+ * causal: 0 or 1.  scale: any finite value (else SDPA_ERR_INVALID_ARG).  A negative
+ * scale is applied by negating Q inside the S = Q K^T product (the instruction's
+ * negate-A bit), so the online softmax always works with |scale|; scale == 0 gives every
+ * visible key weight 1 / (number of visible keys) and LSE = ln(number of visible keys).
  * Every pointer 16-byte aligned (TMA), else SDPA_ERR_MISALIGNED.
  * Arithmetic: S = Q K^T and O += P V on the tensor cores with fp32
  * accumulation; softmax in fp32 with P rounded to bf16; O rounded to bf16
@@ -151,7 +152,11 @@ SDPA_API int sdpa_decode(const void* Q, const void* K, const void* V, const int*
  *    returns SDPA_ERR_WORKSPACE before launching anything.
  *  - Set-up: the first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current.  Make that first call on
- *    every device before any stream capture begins.
+ *    every device before any stream capture begins.  Later calls on a stream that
+ *    is not capturing look the address up again (it allocates nothing), so a device
+ *    reset that reloads the library's module never leaves a stale address behind;
+ *    calls on a capturing stream use the address of the last call outside capture,
+ *    so after a device reset make one call outside capture before capturing again.
  *  - Sharing: every call uses the same array and it keeps the last call's
  *    contents.  Nothing in it needs to start at zero (each call writes every
  *    partial it reads).  Calls whose work overlaps on the GPU (other streams,
@@ -181,7 +186,7 @@ SDPA_API size_t sdpa_bwd_workspace_size(int batch, int heads, int n_q);
  * Nothing of size n_q x n_kv is written; each gradient is written once.
  * Q, O, dO, dQ [batch, heads, n_q, d]; K, V, dK, dV [batch, heads, n_kv, d]; all
  * __nv_bfloat16, contiguous, 16-byte aligned.  LSE [batch, heads, n_q] float as sdpa_fwd wrote
- * it (required).  d_k == d_v in {64, 128}; scale > 0 and causal as in the forward call.
+ * it (required).  d_k == d_v in {64, 128}; scale (any finite value) and causal as in the forward call.
  * workspace: caller-owned device memory of sdpa_bwd_workspace_size bytes (scratch, rewritten
  * by every call: calls that may run at the same time need separate workspaces).
  * Rows whose window held no key (causal, n_q > n_kv) contribute nothing and get dQ = 0.

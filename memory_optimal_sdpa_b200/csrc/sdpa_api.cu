@@ -114,7 +114,8 @@ int launch_prefill(const void* Q, const void* K, const void* V, void* O, float* 
   p.n_kv = n_kv;
   p.bh_count = bh;
   p.n_pairs = (n_q + 255) / 256;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = std::fabs(scale) * 1.4426950408889634f;
+  p.negate_s = scale < 0.f ? 1 : 0;
   p.win_left = win_left;
   p.win_right = win_right;
   // persistent: one CTA per SM (at most one per work unit), each striding over the units
@@ -147,7 +148,7 @@ extern "C" int sdpa_fwd(const void* Q, const void* K, const void* V, void* O, fl
                         void* stream) {
   if (batch < 0 || heads < 0 || n_q < 0 || n_kv < 1 || (causal != 0 && causal != 1) || !std::isfinite(scale))
     return SDPA_ERR_INVALID_ARG;
-  if (d_k != d_v || (d_k != 64 && d_k != 128) || !(scale > 0.f)) return SDPA_ERR_UNSUPPORTED;
+  if (d_k != d_v || (d_k != 64 && d_k != 128)) return SDPA_ERR_UNSUPPORTED;
   if (batch == 0 || heads == 0 || n_q == 0) return SDPA_OK;
   if (!Q || !K || !V || !O) return SDPA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (LSE && !aligned4(LSE)))
@@ -169,7 +170,7 @@ extern "C" int sdpa_fwd_window(const void* Q, const void* K, const void* V, void
                                int window_right, void* stream) {
   if (batch < 0 || heads < 0 || n_q < 0 || n_kv < 1 || window_left < -1 || window_right < -1 || !std::isfinite(scale))
     return SDPA_ERR_INVALID_ARG;
-  if (d_k != d_v || (d_k != 64 && d_k != 128) || !(scale > 0.f)) return SDPA_ERR_UNSUPPORTED;
+  if (d_k != d_v || (d_k != 64 && d_k != 128)) return SDPA_ERR_UNSUPPORTED;
   if (batch == 0 || heads == 0 || n_q == 0) return SDPA_OK;
   if (!Q || !K || !V || !O) return SDPA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (LSE && !aligned4(LSE)))
@@ -272,8 +273,10 @@ constexpr int kMaxDevices = 64;
 std::mutex g_static_scratch_mutex;
 float* g_static_scratch_ptr[kMaxDevices];
 
-// Device address of the scratch array on the current device (looked up once per device).
-float* static_scratch_for_current_device(int* status) {
+// Device address of the scratch array on the current device.  Looked up on the first call on
+// each device, and again on every call whose stream is not capturing (so a device reset that
+// reloads this module cannot leave a stale address); a capturing stream reuses the last one.
+float* static_scratch_for_current_device(cudaStream_t stream, int* status) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -284,8 +287,13 @@ float* static_scratch_for_current_device(int* status) {
     *status = SDPA_ERR_UNSUPPORTED;
     return nullptr;
   }
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess) {
+    (void)cudaGetLastError();  // e.g. the legacy stream while another stream captures: treat as capturing
+    capture = cudaStreamCaptureStatusActive;
+  }
   std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
-  if (!g_static_scratch_ptr[dev]) {
+  if (!g_static_scratch_ptr[dev] || capture == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_static_scratch);
     if (e != cudaSuccess || !p) {
@@ -319,7 +327,7 @@ extern "C" int sdpa_decode_noalloc(const void* Q, const void* K, const void* V, 
   }
   if (int e = check_device()) return e;
   int status = SDPA_OK;
-  float* scratch = static_scratch_for_current_device(&status);
+  float* scratch = static_scratch_for_current_device((cudaStream_t)stream, &status);
   if (!scratch) return status;
   sdpa::DecodeParams p;
   p.Q = (const __nv_bfloat16*)Q;
@@ -519,7 +527,7 @@ extern "C" int sdpa_bwd(const void* Q, const void* K, const void* V, const void*
                         void* dQ, void* dK, void* dV, int batch, int heads, int n_q, int n_kv, int d_k, int d_v,
                         float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
   if (batch < 0 || heads < 0 || n_q < 0 || n_kv < 1 || !std::isfinite(scale)) return SDPA_ERR_INVALID_ARG;
-  if (d_k != d_v || (d_k != 64 && d_k != 128) || !(scale > 0.f)) return SDPA_ERR_UNSUPPORTED;
+  if (d_k != d_v || (d_k != 64 && d_k != 128)) return SDPA_ERR_UNSUPPORTED;
   if (batch == 0 || heads == 0 || n_q == 0) return SDPA_OK;
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return SDPA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned4(LSE) ||

@@ -1,6 +1,6 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features the
-// prefill kernel uses: mbarriers with time-bounded waits, TMA tile loads (no
-// cluster multicast anywhere), and the 5th-generation tensor core interface
+// prefill kernel uses: mbarriers with time-bounded waits, TMA tile loads into the
+// issuing CTA's own shared memory, and the 5th-generation tensor core interface
 // (tcgen05: TMEM allocation, MMA with shared-memory descriptors or a TMEM
 // A operand, commit, TMEM loads/stores and their fences).
 #pragma once

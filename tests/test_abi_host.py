@@ -67,8 +67,10 @@ def test_fwd_argument_errors(sdpa):
     assert fwd(sdpa, scale=float("inf")) == sdpa.SDPA_ERR_INVALID_ARG
     assert fwd(sdpa, dk=96, dv=96) == sdpa.SDPA_ERR_UNSUPPORTED
     assert fwd(sdpa, dk=64, dv=128) == sdpa.SDPA_ERR_UNSUPPORTED
-    assert fwd(sdpa, scale=0.0) == sdpa.SDPA_ERR_UNSUPPORTED
-    assert fwd(sdpa, scale=-0.5) == sdpa.SDPA_ERR_UNSUPPORTED
+    # any finite scale passes the argument checks (zero and negative included): the next
+    # check to fail is the planted misalignment, not the scale
+    assert fwd(sdpa, scale=0.0, O=P + 2) == sdpa.SDPA_ERR_MISALIGNED
+    assert fwd(sdpa, scale=-0.5, K=P + 8) == sdpa.SDPA_ERR_MISALIGNED
     assert fwd(sdpa, K=P + 8) == sdpa.SDPA_ERR_MISALIGNED
     assert fwd(sdpa, O=P + 2) == sdpa.SDPA_ERR_MISALIGNED
     assert fwd(sdpa, LSE=P + 2) == sdpa.SDPA_ERR_MISALIGNED
@@ -87,6 +89,7 @@ def test_fwd_window_argument_errors(sdpa):
     assert f(Q=None) == sdpa.SDPA_ERR_INVALID_ARG
     assert f(dk=96, dv=96) == sdpa.SDPA_ERR_UNSUPPORTED
     assert f(V=P + 2) == sdpa.SDPA_ERR_MISALIGNED
+    assert f(V=P + 2, scale=-0.25) == sdpa.SDPA_ERR_MISALIGNED and f(V=P + 2, scale=0.0) == sdpa.SDPA_ERR_MISALIGNED
     assert f(Q=None, K=None, V=None, O=None, nq=0) == sdpa.SDPA_OK
 
 
@@ -162,7 +165,8 @@ def test_bwd_workspace_and_errors(sdpa):
     assert call(args(dO=None)) == sdpa.SDPA_ERR_INVALID_ARG
     assert call(args(nkv=0)) == sdpa.SDPA_ERR_INVALID_ARG
     assert call(args(dk=128, dv=64)) == sdpa.SDPA_ERR_UNSUPPORTED
-    assert call(args(scale=-1.0)) == sdpa.SDPA_ERR_UNSUPPORTED
+    assert call(args(scale=-1.0, dQ=P + 2)) == sdpa.SDPA_ERR_MISALIGNED
+    assert call(args(scale=0.0, dK=P + 2)) == sdpa.SDPA_ERR_MISALIGNED
     assert call(args(dQ=P + 2)) == sdpa.SDPA_ERR_MISALIGNED
     assert call(args(nq=0)) == sdpa.SDPA_OK
 

@@ -52,7 +52,8 @@ def grad_bounds(q, k, v, do, scale, causal):
     ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
     delta = 2.0 ** -9 * np.abs(do * o).sum(axis=1, keepdims=True)
     w = 2.0 ** -8 * np.abs(ds) + p * delta
-    return (scale * (w @ np.abs(k)), scale * (w.T @ np.abs(q)), 2.0 ** -8 * (p.T @ np.abs(do)))
+    a = abs(scale)
+    return (a * (w @ np.abs(k)), a * (w.T @ np.abs(q)), 2.0 ** -8 * (p.T @ np.abs(do)))
 
 
 def check_grad(G, G_ref, bound, what):
@@ -201,3 +202,28 @@ def test_bwd_complete_for_work_queued_behind_it(sdpa, cuda_device):
                 assert torch.equal(c, g), "%s read behind sdpa_bwd differs (causal=%s)" % (name, causal)
             assert dv.abs().sum().item() > 0
     assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.125, -0.0883883461356163])
+@pytest.mark.parametrize("B,H,n_q,n_kv,d,causal", [(1, 2, 256, 256, 64, True), (1, 2, 300, 200, 128, False),
+                                                    (1, 2, 333, 333, 128, True), (1, 2, 200, 333, 64, False)])
+def test_bwd_zero_and_negative_scale(sdpa, cuda_device, B, H, n_q, n_kv, d, causal, scale):
+    # The gradient formulas hold for any finite scale (the MoA article's definition fixes the
+    # scale only by convention): scale = 0 makes P uniform over the visible keys and dQ = dK = 0;
+    # a negative scale flips the logits.  The forward feeding this is the same call.
+    seed = 900 + n_q + 3 * n_kv + d + int(causal)
+    q = si.fill_host((B, H, n_q, d), seed, 0)
+    k = si.fill_host((B, H, n_kv, d), seed, 1)
+    v = si.fill_host((B, H, n_kv, d), seed, 2)
+    do = si.fill_host((B, H, n_q, d), seed, si.STREAM_DO)
+    scale = float(np.float32(scale))
+    dq, dk, dv = run_bwd(sdpa, cuda_device, q, k, v, do, causal, scale)
+    qf, kf, vf, dof = (si.bf16_bits_to_f32(x) for x in (q, k, v, do))
+    dQ, dK, dV = oracle.sdpa_backward(qf, kf, vf, dof, scale, causal)
+    for b in range(B):
+        for h in range(H):
+            tag = "%s scale=%g b=%d h=%d" % ((B, H, n_q, n_kv, d, causal), scale, b, h)
+            check_slice(dq[b, h], dk[b, h], dv[b, h], dQ[b, h], dK[b, h], dV[b, h], qf[b, h], kf[b, h], vf[b, h],
+                        dof[b, h], scale, causal, tag)
+    if scale == 0.0:
+        assert (dq == 0).all() and (dk == 0).all()

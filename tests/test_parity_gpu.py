@@ -136,6 +136,45 @@ def test_prefill_identity_values_give_probabilities(sdpa, cuda_device):
             assert (np.abs(O - P) <= 2 ** -7 * P + 1e-6).all(), "d=%d causal=%d" % (d, causal)
 
 
+ANY_SCALE = [
+    # (n_q, n_kv, d, mode): mode full, causal, or a (left, right) window
+    (256, 256, 64, "full"), (300, 333, 64, "causal"), (513, 700, 128, "causal"), (640, 640, 128, "full"),
+    (333, 300, 128, "causal"), (700, 700, 64, (100, 0)), (600, 600, 128, (200, 50)),
+]
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.125, -0.0883883461356163, -1.5])
+@pytest.mark.parametrize("n_q,n_kv,d,mode", ANY_SCALE)
+def test_prefill_zero_and_negative_scale(sdpa, cuda_device, n_q, n_kv, d, mode, scale):
+    # The definition fixes the scale only by convention (MoA article, "DNF derivation"), so any
+    # finite value is accepted: 0 gives the mean of the visible V rows and LSE = ln(count); a
+    # negative scale is carried by the S product itself (negated A operand).  -1.5 drives the
+    # logits far past the lazy-rescale threshold, so the running maximum moves too.
+    import torch
+    B, H = 1, 2
+    seed = 700 + n_q + 5 * n_kv + d
+    q = si.fill_host((B, H, n_q, d), seed, 0)
+    k = si.fill_host((B, H, n_kv, d), seed, 1)
+    v = si.fill_host((B, H, n_kv, d), seed, 2)
+    scale = float(np.float32(scale))
+    tq, tk, tv = (W.to_torch(x, cuda_device) for x in (q, k, v))
+    o_flat, o = _nan_buffer((B, H, n_q, d), torch.bfloat16, cuda_device, 128 * d)
+    l_flat, lse = _nan_buffer((B, H, n_q), torch.float32, cuda_device, 256)
+    qf, kf, vf = (si.bf16_bits_to_f32(x) for x in (q, k, v))
+    if isinstance(mode, tuple):
+        sdpa.fwd_window(tq, tk, tv, mode[0], mode[1], scale=scale, o=o, lse=lse)
+        O_ref, L_ref = oracle.sdpa_rows_window(qf, kf, vf, scale, mode[0], mode[1])
+    else:
+        sdpa.fwd(tq, tk, tv, causal=(mode == "causal"), scale=scale, o=o, lse=lse)
+        O_ref, L_ref = oracle.sdpa_rows(qf, kf, vf, scale, mode == "causal")
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    check_bf16(o.float().cpu().numpy(), O_ref, lse.cpu().numpy(), L_ref,
+               "scale %g %s" % (scale, (n_q, n_kv, d, mode)))
+    assert torch.isnan(o_flat[o.numel():]).all() and torch.isnan(l_flat[lse.numel():]).all()
+    if scale == 0.0 and mode == "full":  # closed form: every row is the mean of V, LSE = ln(n_kv)
+        assert np.abs(lse.cpu().numpy() - math.log(n_kv)).max() <= 1e-5
+
+
 @pytest.mark.parametrize("d,causal", [(64, False), (64, True), (128, False), (128, True)])
 def test_prefill_rescale_every_tile(sdpa, cuda_device, d, causal):
     # Keys grow tile by tile (128-key tiles), so every row's maximum rises by far more than the
