@@ -1,20 +1,27 @@
 """Benchmark: exact attention on B200 through the library's C ABI, one JSON line on rank 0.
 
-Headline step (default workload cfg2): one bf16 prefill, batch 4, 16 heads,
-n_q = n_kv = 2048, d = 64, scale 1/8, run non-causal AND causal -- both
-launches of the tcgen05 prefill kernel -- over inputs resident in HBM.
-value = algorithmic TFLOP/s (2 matmuls x 2 FLOP per multiply-add, causal
-halved).  L2 is flushed (256 MiB write) before every timed step; each step is
-timed with CUDA events on the launching stream and the flush is excluded.
+Headline step (default workload cfg4, the largest single-GPU prefill): one bf16
+prefill launch, batch 1, 8 heads, n_q = n_kv = 32768, d = 128, Q,K ~ N(0, 2.5^2),
+V ~ N(0,1), scale 1/sqrt(128), non-causal, over inputs resident in HBM.
+value = algorithmic TFLOP/s (two matmuls, 2 FLOP per multiply-add, causal
+halved).  L2 is flushed (256 MiB write) before every timed launch; each launch
+is timed with CUDA events on the launching stream and the flush is excluded.
 
 The line also carries:
-  roofline     the prefill kernel's achieved TFLOP/s against the measured bf16 peak
-  decode       the decode workload (64 x 32 heads, cache 16384, lengths U{1024..16384},
-               d = 128) in GB/s of algorithmic bytes against the measured HBM copy rate
-  e2e          the same step through the public API from pinned host buffers
-               (host->device inputs and device->host outputs inside the timed region)
-  cpu_baseline the CPU oracle on a bounded sample of rows of the same workload
-  clocks       nvidia-smi SM clocks and throttle reasons sampled during the timed region
+  roofline      the headline kernel's achieved TFLOP/s against the measured bf16 peak, and
+                against the spec dense-bf16 figure
+  prefill_legs  the other prefill workloads, each in its own timed loop (at least
+                --leg-seconds of launches) with its own roofline: cfg2 (d = 64, 4 x 16 heads,
+                n = 2048) non-causal and causal, cfg3 (d = 128 causal, 32 heads, n = 8192),
+                cfg3w (cfg3 under a 512-key causal window)
+  backward      dQ, dK, dV of cfg2, cfg2 causal and cfg3
+  decode        the decode workload (64 x 32 heads, cache 16384, lengths U{1024..16384},
+                d = 128) in GB/s of algorithmic bytes against the measured HBM copy rate;
+                decode_gqa the same with 64 query heads over 8 key/value heads
+  e2e           the headline step through the public API from pinned host buffers
+                (host->device inputs and device->host outputs inside the timed region)
+  cpu_baseline  the CPU oracle on a bounded sample of rows of the headline workload
+  clocks        nvidia-smi SM clocks and throttle reasons sampled during the timed region
 
 Multi-GPU: `torchrun --nproc-per-node N bench.py --gpus N`: every rank runs an
 independent replica (attention over independent (batch, head) slices needs no
@@ -38,11 +45,24 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures (dense bf16 tensor, HBM3e), the spec denominators reported beside the measured ones
+SPEC = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 PREFILL_SOURCES = ["memory_optimal_sdpa_b200/csrc/prefill_bf16.cuh", "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
 DECODE_SOURCES = ["memory_optimal_sdpa_b200/csrc/decode.cuh"]
 BWD_SOURCES = ["memory_optimal_sdpa_b200/csrc/backward.cuh", "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
 GQA_SOURCES = ["memory_optimal_sdpa_b200/csrc/decode_gqa.cuh", "memory_optimal_sdpa_b200/csrc/decode.cuh",
                "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
+PREFILL_WORKLOADS = ["cfg4", "cfg3", "cfg2", "cfg2c", "cfg3w"]
+METRIC = "attention fwd TFLOP/s (prefill) & decode HBM GB/s, as % of B200 roofline"
+DESCRIBE = {
+    "cfg2": "cfg2: prefill bf16 batch 4 x 16 heads, n_q = n_kv = 2048, d_k = d_v = 64, scale 1/8, non-causal",
+    "cfg2c": "cfg2c: prefill bf16 batch 4 x 16 heads, n_q = n_kv = 2048, d_k = d_v = 64, scale 1/8, causal",
+    "cfg3": "cfg3: prefill bf16 batch 1 x 32 heads, n_q = n_kv = 8192, d_k = d_v = 128, scale 1/sqrt(128), causal, "
+            "V ~ U(-1,1)",
+    "cfg4": "cfg4: prefill bf16 batch 1 x 8 heads, n_q = n_kv = 32768, d_k = d_v = 128, scale 1/sqrt(128), "
+            "non-causal, Q,K ~ N(0, 2.5^2)",
+    "cfg3w": "cfg3w: cfg3 under a causal local window of 512 keys (window_left 511, window_right 0)",
+}
 
 
 def load_peaks():
@@ -75,32 +95,33 @@ def profiled_traffic(summary, paths):
     if fields.get("source_digest") != source_digest(paths):
         return None
     try:
-        return float(fields["dram_bytes_per_launch_full_workload"])
-    except (KeyError, ValueError):
+        return float(fields["dram_bytes_per_launch_full_workload"].split()[0])
+    except (KeyError, ValueError, IndexError):
         return None
 
 
 class ClockSampler:
-    """nvidia-smi SM clocks, utilisation and throttle reasons, sampled every 100 ms while running.
+    """nvidia-smi SM clocks, utilisation and throttle reasons, sampled every 20 ms while running.
 
-    summary(t0, t1) reports the samples taken inside [t0, t1] (host wall clock; the timed
-    region) when there are any, else the samples of the whole window during which the GPU
-    was busy (utilisation > 0), and says which.
+    summary(t0, t1) reports the samples taken inside [t0, t1] (host wall clock; a timed region)
+    when there are any, else the samples of the whole window during which the GPU was busy
+    (utilisation > 0), and says which.
     """
     QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,utilization.gpu,clocks_event_reasons.hw_slowdown,"
              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
              "clocks_event_reasons.sw_power_cap")
     NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, index):
+    def __init__(self, index, period_ms=20):
         self.index = index
+        self.period_ms = period_ms
         self.proc = None
         self.samples = []  # (unix time, sm_mhz, max_mhz, util, reasons)
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -124,7 +145,7 @@ class ClockSampler:
 
     def __exit__(self, *exc):
         if self.proc:
-            time.sleep(0.25)  # let the last sample land
+            time.sleep(0.1)  # let the last sample land
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -133,7 +154,7 @@ class ClockSampler:
             self.thread.join(timeout=2)
 
     def summary(self, t0=None, t1=None):
-        inside = [x for x in self.samples if t0 is not None and t0 - 0.05 <= x[0] <= t1 + 0.05]
+        inside = [x for x in self.samples if t0 is not None and t0 - 0.01 <= x[0] <= t1 + 0.01]
         chosen, where = inside, "timed region"
         if not chosen:
             chosen, where = [x for x in self.samples if x[3] > 0], "busy samples of the bench window"
@@ -141,7 +162,8 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "from": "none"}
         reasons = sorted(set().union(*(x[4] for x in chosen)))
         return {"sm_mhz": float(np.median([x[1] for x in chosen])), "sm_max_mhz": chosen[-1][2],
-                "reasons": reasons, "samples": len(chosen), "from": where}
+                "sm_mhz_min": float(min(x[1] for x in chosen)), "reasons": reasons, "samples": len(chosen),
+                "from": where, "period_ms": self.period_ms}
 
 
 # ---------------------------------------------------------------------------------------------- distributed
@@ -172,7 +194,7 @@ def barrier():
 
 # ------------------------------------------------------------------------------------------------ oracle leg
 def oracle_rate(w_list, seconds_target, seed=0):
-    """CPU oracle on sampled rows of the workloads; returns (TFLOP/s, cores, description)."""
+    """CPU oracle on sampled rows of the workloads; returns (TFLOP/s, cores, description, seconds)."""
     import oracle
     import seeded_inputs as si
     from seeded_inputs import workloads as W
@@ -193,8 +215,8 @@ def oracle_rate(w_list, seconds_target, seed=0):
             flops += float(vis.sum()) * 2 * (w.d + w.d) * w.batch * w.heads
         return flops, time.perf_counter() - t0
 
-    f, t = run(8)
-    per_row = t / (8 * w0.batch * w0.heads * len(w_list))
+    f, t = run(2)
+    per_row = t / (2 * w0.batch * w0.heads * len(w_list))
     rows = int(max(2, min(w0.n_q, seconds_target / max(per_row, 1e-9) / (w0.batch * w0.heads * len(w_list)))))
     f, t = run(rows)
     desc = "%d sampled query rows per head of each of %s (oracle, double precision)" % (
@@ -227,97 +249,93 @@ def standard_bytes(w):
     return w.bytes() + w.batch * w.heads * w.n_q * w.n_kv * 12
 
 
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
+def tensor_roofline(kernel, flops, nbytes, t, peaks, peak_kind, traffic, note):
+    """Roofline object of a tensor-pipe-bound launch: algorithmic FLOPs / mean launch time against the
+    measured burst bf16 peak (the kernel is timed alone) and against the spec dense-bf16 figure."""
+    peak = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    a = flops / t / 1e12
+    return {"kernel": kernel, "bound": "tensor", "achieved": round(a, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(a / peak, 4), "peak_kind": peak_kind + " burst bf16 (kernel timed alone)",
+            "spec_peak": SPEC["bf16_tflops"], "spec_frac": round(a / SPEC["bf16_tflops"], 4),
+            "sustained_peak": peaks.get("bf16_tflops_sustained"),
+            "sustained_frac": (round(a / peaks["bf16_tflops_sustained"], 4) if peaks.get("bf16_tflops_sustained")
+                               else None),
+            "algorithmic_flop_per_launch": float(flops), "algorithmic_bytes_per_launch": float(nbytes),
+            "traffic": traffic,
+            "traffic_over_algorithmic_bytes": None if traffic is None else round(traffic / nbytes, 3),
+            "traffic_source": note}
 
-    import memory_optimal_sdpa_b200 as sdpa
-    import seeded_inputs as si
+
+def hbm_roofline(kernel, nbytes, t, peaks, peak_kind, traffic):
+    peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    g = nbytes / t / 1e9
+    return {"kernel": kernel, "bound": "hbm", "achieved": round(g, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(g / peak, 4), "peak_kind": peak_kind + " HBM copy", "spec_peak": SPEC["hbm_gbs"],
+            "spec_frac": round(g / SPEC["hbm_gbs"], 4), "traffic": traffic, "algorithmic_bytes": float(nbytes)}
+
+
+def workload(name):
     from seeded_inputs import workloads as W
+    return getattr(W, name.upper())
 
-    rank, local_rank, world = dist_env()
-    if world != args.gpus:
-        raise SystemExit("--gpus %d but WORLD_SIZE=%d: launch N>1 with torchrun" % (args.gpus, world))
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    peaks, peak_kind = load_peaks()
-    w_nc = W.CFG2 if args.workload == "cfg2" else getattr(W, args.workload.upper())
-    works = [w_nc, w_nc.with_causal(True)] if args.workload == "cfg2" else [w_nc]
+def kernel_name(w):
+    mask = 2 if w.window is not None else int(w.causal)
+    return "sdpa_fwd_bf16_kernel<%d,%d>" % (w.d, mask)
 
-    # Inputs: generated on the host (seeded), copied once; resident in HBM for the device-timed region.
-    host = W.prefill_host(w_nc)
-    q, k, v = (W.to_torch(host[n], dev) for n in ("q", "k", "v"))
-    outs = [(torch.empty_like(q), torch.empty((w_nc.batch, w_nc.heads, w_nc.n_q), dtype=torch.float32, device=dev))
-            for _ in works]
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
 
-    def call(w, qq, kk, vv, o, lse):
-        if w.window is not None:
-            sdpa.fwd_window(qq, kk, vv, w.window[0], w.window[1], scale=w.scale_f32, o=o, lse=lse, stream=stream)
-        else:
-            sdpa.fwd(qq, kk, vv, causal=w.causal, scale=w.scale_f32, o=o, lse=lse, stream=stream)
+class PrefillInputs:
+    """Seeded inputs of a prefill workload, resident on the device, and its output buffers."""
 
-    def step(qq=q, kk=k, vv=v):
-        for w, (o, lse) in zip(works, outs):
-            call(w, qq, kk, vv, o, lse)
+    def __init__(self, w, dev):
+        import torch
+        from seeded_inputs import workloads as W
+        self.w = w
+        self.host = W.prefill_host(w)
+        self.q, self.k, self.v = (W.to_torch(self.host[n], dev) for n in ("q", "k", "v"))
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((w.batch, w.heads, w.n_q), dtype=torch.float32, device=dev)
 
-    clocks = ClockSampler(local_rank).__enter__()  # sampled from warm-up through the end-to-end loop
-    time.sleep(0.3)
-    for _ in range(args.warmup):
-        step()
-    if sdpa.get_last_device_error() != sdpa.SDPA_OK:
-        raise SystemExit("device error during warm-up")
 
-    # ---- device-timed region: K steps, L2 flushed before each (flush not timed)
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in works]
-          for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
-    t_wall0 = time.time()
-    for s in range(args.steps):
+def prefill_call(sdpa, w, q, k, v, o, lse, stream):
+    if w.window is not None:
+        sdpa.fwd_window(q, k, v, w.window[0], w.window[1], scale=w.scale_f32, o=o, lse=lse, stream=stream)
+    else:
+        sdpa.fwd(q, k, v, causal=w.causal, scale=w.scale_f32, o=o, lse=lse, stream=stream)
+
+
+def timed_launches(call, n, flush, stream):
+    """n launches, each preceded by an (untimed) L2 flush and bracketed by CUDA events on `stream`;
+    returns the per-launch seconds."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in ev:
         flush.zero_()
-        for (a, b), w, (o, lse) in zip(ev[s], works, outs):
-            a.record(stream)
-            call(w, q, k, v, o, lse)
-            b.record(stream)
+        a.record(stream)
+        call()
+        b.record(stream)
     torch.cuda.synchronize()
-    t_wall1 = time.time()
-    barrier()
-    per_launch = np.array([[a.elapsed_time(b) for (a, b) in row] for row in ev]) / 1e3  # seconds [step, launch]
-    local_t = float(per_launch.sum())
-    step_flops = sum(w.flops() for w in works)
-    t_max, units = aggregate(local_t, step_flops * args.steps)
-    value = units / t_max / 1e12
-    if sdpa.get_last_device_error() != sdpa.SDPA_OK:
-        raise SystemExit("device error in the timed region")
+    return np.array([a.elapsed_time(b) for a, b in ev]) / 1e3
 
-    # roofline of the dominant kernel (the first launch of the step): algorithmic FLOPs / mean launch time
-    peak_tf = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
-    dom = works[0]
-    t_dom = float(per_launch[:, 0].mean())
-    achieved = dom.flops() / t_dom / 1e12
-    roof = {"kernel": "sdpa_fwd_bf16_kernel<%d,%d> (%s)" % (dom.d, int(dom.causal), dom.name), "bound": "tensor",
-            "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
-            "peak_kind": peak_kind + " burst bf16 (kernel timed alone)",
-            "algorithmic_flop_per_launch": dom.flops(),
-            "traffic": profiled_traffic("prefill_%s_dram.txt" % dom.name, PREFILL_SOURCES),
-            "per_launch_ms": {w.name: round(float(per_launch[:, i].mean()) * 1e3, 4) for i, w in enumerate(works)},
-            "per_launch_tflops": {w.name: round(w.flops() / float(per_launch[:, i].mean()) / 1e12, 1)
-                                  for i, w in enumerate(works)}}
 
-    # ---- end to end through the public API: pinned host inputs -> device -> pinned host outputs.
-    # Every step copies all of its inputs in and all of its outputs out; the copies of neighbouring
-    # steps run on their own streams (double-buffered device tensors), overlapping this step's kernels.
-    hq, hk, hv = (torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v"))
-    dins = [tuple(torch.empty_like(x) for x in (q, k, v)) for _ in range(2)]
-    douts = [[(torch.empty_like(o), torch.empty_like(l)) for o, l in outs] for _ in range(2)]
-    houts = [[(torch.empty(o.shape, dtype=o.dtype).pin_memory(), torch.empty(l.shape, dtype=l.dtype).pin_memory())
-              for o, l in outs] for _ in range(2)]
+def launches_for(call, flush, stream, seconds, minimum):
+    """Launch count that fills about `seconds` of device time (at least `minimum`)."""
+    t = float(np.median(timed_launches(call, 3, flush, stream)))
+    return max(minimum, int(math.ceil(seconds / max(t, 1e-7))))
+
+
+def run_e2e(sdpa, w, inp, stream, steps):
+    """The headline step end to end through the public API: pinned host inputs -> device -> pinned host
+    outputs.  Every step copies all of its inputs in and all of its outputs out; the copies of
+    neighbouring steps run on their own streams (double-buffered device tensors), overlapping this
+    step's kernel.  Returns (seconds for `steps` steps on this rank, h2d bytes, d2h bytes per step)."""
+    import torch
+    hq, hk, hv = (torch.from_numpy(inp.host[n].view(np.int16)).view(torch.bfloat16).pin_memory()
+                  for n in ("q", "k", "v"))
+    dins = [tuple(torch.empty_like(x) for x in (inp.q, inp.k, inp.v)) for _ in range(2)]
+    douts = [(torch.empty_like(inp.o), torch.empty_like(inp.lse)) for _ in range(2)]
+    houts = [(torch.empty(inp.o.shape, dtype=inp.o.dtype).pin_memory(),
+              torch.empty(inp.lse.shape, dtype=inp.lse.dtype).pin_memory()) for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
     def e2e_run(n):
@@ -341,16 +359,16 @@ def run_ours(args):
                 stream.wait_event(ev_in[j])
                 if j >= 2:
                     stream.wait_event(ev_out[j - 2])
-                for w, (o, lse) in zip(works, douts[j % 2]):
-                    call(w, *dins[j % 2], o, lse)
+                o, lse = douts[j % 2]
+                prefill_call(sdpa, w, *dins[j % 2], o, lse, stream)
                 ev_comp[j].record(stream)
             m = i - 2
             if 0 <= m < n:  # copy out step m
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(ev_comp[m])
-                    for (o, l), (po, pl) in zip(douts[m % 2], houts[m % 2]):
-                        po.copy_(o, non_blocking=True)
-                        pl.copy_(l, non_blocking=True)
+                    (o, l), (po, pl) = douts[m % 2], houts[m % 2]
+                    po.copy_(o, non_blocking=True)
+                    pl.copy_(l, non_blocking=True)
                     ev_out[m].record(s_out)
         t1.record(s_out)
         torch.cuda.synchronize()
@@ -358,107 +376,68 @@ def run_ours(args):
 
     e2e_run(3)
     barrier()
-    e_local = e2e_run(args.steps)
-    clocks.__exit__(None, None, None)
-    e_max, e_units = aggregate(e_local, step_flops * args.steps)
+    t = e2e_run(steps)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
-    d2h = sum(po.numel() * po.element_size() + pl.numel() * pl.element_size() for po, pl in houts[0])
-    e2e = {"value": round(e_units / e_max / 1e12, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h,
-           "schedule": "steps pipelined: step i+1's inputs copied in and step i-1's outputs copied out "
-                       "(pinned host memory, own streams) while step i computes"}
-    del hq, hk, hv, houts, dins, douts
-
-    # ---- backward pass on the same workload (its own sub-benchmark)
-    backward = None if args.skip_backward else run_backward(args, sdpa, si, W, works, q, k, v, outs, stream, flush,
-                                                             peaks, peak_kind)
-
-    # ---- decode workload (HBM-bound), its own roofline
-    decode = None if args.skip_decode else run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind)
-    decode_gqa = (None if args.skip_decode else
-                  run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, grouped=True))
-
-    line = {
-        "metric": "attention fwd TFLOP/s (prefill) & decode HBM GB/s, as % of B200 roofline",
-        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(t_max / args.steps * 1e3, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64/Box-Muller, bf16 RNE)",
-        "config": {"workload": "cfg2: prefill bf16 batch 4 x 16 heads, n_q = n_kv = 2048, d_k = d_v = 64, scale 1/8, "
-                               "non-causal + causal per step" if args.workload == "cfg2" else args.workload,
-                   "global_batch": w_nc.batch * world, "seq_len": w_nc.n_q, "heads": w_nc.heads, "head_dim": w_nc.d,
-                   "parallelism": "replicas x%d (independent heads, no collective)" % world,
-                   "l2": "flushed before every timed step (256 MiB write, not timed)"},
-        "roofline": roof,
-        "cost_model": {w.name: cost_model(w.flops(), w.bytes(), float(per_launch[:, i].mean()), peaks, standard_bytes(w))
-                       for i, w in enumerate(works)},
-        "gpu_launches": args.steps * len(works),
-        "e2e": e2e,
-        "clocks": clocks.summary(t_wall0, t_wall1),
-    }
-    if backward is not None:
-        line["backward"] = backward
-    if decode is not None:
-        line["decode"] = decode
-    if decode_gqa is not None:
-        line["decode_gqa"] = decode_gqa
-    if rank == 0 and world == 1 and not args.skip_cpu:
-        rate, cores, desc, secs = oracle_rate(works, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": round(rate, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                "sample": desc, "seconds": round(secs, 2)}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    d2h = sum(x.numel() * x.element_size() for x in houts[0])
+    return t, h2d, d2h
 
 
-def run_backward(args, sdpa, si, W, works, q, k, v, outs, stream, flush, peaks, peak_kind):
-    """dQ, dK, dV of each prefill workload of the step, from the forward's O and LSE.  Algorithmic
-    FLOPs: 2.5x the forward's (five matrix products of the gradient); the kernels execute seven
-    (S and dP are formed in both the dK/dV and the dQ kernel)."""
+def run_prefill_leg(args, sdpa, name, dev, stream, flush, peaks, peak_kind, clocks):
+    w = workload(name)
+    inp = PrefillInputs(w, dev)
+    call = lambda: prefill_call(sdpa, w, inp.q, inp.k, inp.v, inp.o, inp.lse, stream)
+    for _ in range(args.warmup):
+        call()
+    n = launches_for(call, flush, stream, args.leg_seconds, args.steps)
+    t0 = time.time()
+    per = timed_launches(call, n, flush, stream)
+    t1 = time.time()
+    if sdpa.get_last_device_error() != sdpa.SDPA_OK:
+        raise SystemExit("device error in prefill leg %s" % name)
+    t = float(per.mean())
+    traffic = profiled_traffic("prefill_%s_dram.txt" % name, PREFILL_SOURCES)
+    return {"workload": DESCRIBE[name], "launches": n, "ms": round(t * 1e3, 4), "ms_min": round(float(per.min()) * 1e3, 4),
+            "value": round(w.flops() / t / 1e12, 2), "unit": "TFLOP/s",
+            "roofline": tensor_roofline(kernel_name(w) + " (%s)" % name, w.flops(), w.bytes(), t, peaks, peak_kind,
+                                        traffic, "profiles/prefill_%s_dram.txt" % name),
+            "cost_model": cost_model(w.flops(), w.bytes(), t, peaks, standard_bytes(w)),
+            "clocks": clocks.summary(t0, t1)}
+
+
+def run_backward(args, sdpa, si, W, name, dev, stream, flush, peaks, peak_kind, clocks):
+    """dQ, dK, dV of a prefill workload from the forward's O and LSE.  Algorithmic FLOPs: 2.5x the
+    forward's (five matrix products of the gradient); the kernels execute 3.5x (S and dP are formed
+    in both the dK/dV and the dQ kernel)."""
     import torch
-    w0 = works[0]
-    do = W.to_torch(si.fill_host((w0.batch, w0.heads, w0.n_q, w0.d), w0.seed, si.STREAM_DO), q.device)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(sdpa.bwd_workspace_size(w0.batch, w0.heads, w0.n_q), dtype=torch.uint8, device=q.device)
-    res = {}
-    for w, (o, lse) in zip(works, outs):
-        if w.window is not None:  # the backward pass takes full or causal attention
-            continue
-        call = lambda: sdpa.bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale_f32, dq=dq, dk=dk, dv=dv,
-                                workspace=ws, stream=stream)
-        for _ in range(max(3, args.warmup)):
-            call()
-        torch.cuda.synchronize()
-        times = []
-        for _ in range(args.steps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            call()
-            b.record(stream)
-            torch.cuda.synchronize()
-            times.append(a.elapsed_time(b) / 1e3)
-        if sdpa.get_last_device_error() != sdpa.SDPA_OK:
-            raise SystemExit("device error in backward")
-        t = float(np.mean(times))
-        flops = 2.5 * w.flops()
-        peak = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
-        res[w.name] = {"value": round(flops / t / 1e12, 1), "unit": "TFLOP/s", "ms": round(t * 1e3, 4),
-                       "gpu_launches_per_call": 3,
-                       "roofline": {"kernel": "sdpa_bwd_pre + sdpa_bwd_dkdv + sdpa_bwd_dq", "bound": "tensor",
-                                    "achieved": round(flops / t / 1e12, 1), "peak": peak, "unit": "TFLOP/s",
-                                    "frac": round(flops / t / 1e12 / peak, 4),
-                                    "peak_kind": peak_kind + " burst bf16", "algorithmic_flop": flops,
-                                    "executed_flop": 3.5 * w.flops(),
-                                    "traffic": (profiled_traffic("backward_cfg2_dram.txt", BWD_SOURCES)
-                                                if w.name == "cfg2" else None),
-                                    "traffic_covers": "dK/dV and dQ kernels (ncu); not the preprocess kernel"}}
-    del dq, dk, dv, ws, do
-    return res
+    w = workload(name)
+    inp = PrefillInputs(w, dev)
+    prefill_call(sdpa, w, inp.q, inp.k, inp.v, inp.o, inp.lse, stream)
+    do = W.to_torch(si.fill_host((w.batch, w.heads, w.n_q, w.d), w.seed, si.STREAM_DO), dev)
+    dq, dk, dv = torch.empty_like(inp.q), torch.empty_like(inp.k), torch.empty_like(inp.v)
+    ws = torch.empty(sdpa.bwd_workspace_size(w.batch, w.heads, w.n_q), dtype=torch.uint8, device=dev)
+    call = lambda: sdpa.bwd(inp.q, inp.k, inp.v, inp.o, do, inp.lse, causal=w.causal, scale=w.scale_f32,
+                            dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
+    for _ in range(args.warmup):
+        call()
+    n = launches_for(call, flush, stream, args.leg_seconds, args.steps)
+    t0 = time.time()
+    per = timed_launches(call, n, flush, stream)
+    t1 = time.time()
+    if sdpa.get_last_device_error() != sdpa.SDPA_OK:
+        raise SystemExit("device error in backward %s" % name)
+    t = float(per.mean())
+    flops = 2.5 * w.flops()
+    nbytes = 2 * w.bytes()  # Q, K, V, O, dO and LSE read; dQ, dK, dV written (dO is O's size)
+    roof = tensor_roofline("sdpa_bwd_pre + sdpa_bwd_dkdv + sdpa_bwd_dq (%s)" % name, flops, nbytes, t, peaks,
+                           peak_kind, profiled_traffic("backward_%s_dram.txt" % name, BWD_SOURCES),
+                           "profiles/backward_%s_dram.txt (dK/dV and dQ kernels)" % name)
+    roof["executed_flop"] = 3.5 * w.flops()
+    return {"workload": DESCRIBE[name], "launches": n, "gpu_launches_per_call": 3, "ms": round(t * 1e3, 4),
+            "value": round(flops / t / 1e12, 1), "unit": "TFLOP/s", "roofline": roof,
+            "clocks": clocks.summary(t0, t1)}
 
 
-def run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, grouped=False):
+def run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, clocks, grouped=False):
     """Decode sub-benchmark: cfg5 (one key/value head per query head) or, grouped, cfg5g."""
     import torch
     w = W.CFG5G if grouped else W.CFG5
@@ -482,23 +461,16 @@ def run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, grouped=
     else:
         ws = torch.empty(sdpa.decode_workspace_size(w.batch, w.heads, w.n_cap, w.d), dtype=torch.uint8, device=dev)
         call = lambda: sdpa.decode(q, kc, vc, tl, scale=w.scale_f32, o=o, lse=lse, workspace=ws, stream=stream)
-    for _ in range(max(3, args.warmup)):
+    for _ in range(args.warmup):
         call()
-    torch.cuda.synchronize()
-    times = []
-    for _ in range(args.steps):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        call()
-        b.record(stream)
-        torch.cuda.synchronize()
-        times.append(a.elapsed_time(b) / 1e3)
+    n = launches_for(call, flush, stream, args.leg_seconds, args.steps)
+    t0 = time.time()
+    per = timed_launches(call, n, flush, stream)
+    t1 = time.time()
     if sdpa.get_last_device_error() != sdpa.SDPA_OK:
         raise SystemExit("device error in decode")
-    t = float(np.mean(times))
+    t = float(per.mean())
     gbs = w.bytes(lens) / t / 1e9
-    peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
     del kc, vc
     torch.cuda.empty_cache()
     heads = ("%d query heads over %d key/value heads" % (w.heads, w.kv_heads)) if grouped else "%d heads" % w.heads
@@ -506,16 +478,124 @@ def run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, grouped=
         kernel, prof, srcs = "sdpa_decode_gqa_kernel<16> + combine", "decode_cfg5g_dram.txt", GQA_SOURCES
     else:
         kernel, prof, srcs = "sdpa_decode_split_kernel + combine", "decode_cfg5_dram.txt", DECODE_SOURCES
+    traffic = None if args.decode_batch != 64 else profiled_traffic(prof, srcs)
     return {"workload": "%s: decode bf16 batch %d x %s, cache 16384, lengths U{1024..16384} (sum %d), d = 128"
                         % (w.name, w.batch, heads, int(lens.sum())),
-            "value": round(gbs, 1), "unit": "GB/s", "ms": round(t * 1e3, 4), "gpu_launches_per_call": 2,
-            "gflops": round(w.flops(lens) / t / 1e9, 1),
+            "launches": n, "value": round(gbs, 1), "unit": "GB/s", "ms": round(t * 1e3, 4),
+            "gpu_launches_per_call": 2, "gflops": round(w.flops(lens) / t / 1e9, 1),
             "cost_model": cost_model(w.flops(lens), w.bytes(lens), t, peaks),
-            "roofline": {"kernel": kernel, "bound": "hbm", "achieved": round(gbs, 1),
-                         "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
-                         "peak_kind": peak_kind + " HBM copy",
-                         "traffic": (None if args.decode_batch != 64 else profiled_traffic(prof, srcs)),
-                         "algorithmic_bytes": w.bytes(lens)}}
+            "roofline": hbm_roofline(kernel, w.bytes(lens), t, peaks, peak_kind, traffic),
+            "clocks": clocks.summary(t0, t1)}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import memory_optimal_sdpa_b200 as sdpa
+    import seeded_inputs as si
+    from seeded_inputs import workloads as W
+
+    rank, local_rank, world = dist_env()
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d: launch N>1 with torchrun" % (args.gpus, world))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    peaks, peak_kind = load_peaks()
+    wh = workload(args.workload)
+    inp = PrefillInputs(wh, dev)  # seeded on the host, copied once: resident in HBM for the timed region
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    call = lambda: prefill_call(sdpa, wh, inp.q, inp.k, inp.v, inp.o, inp.lse, stream)
+
+    clocks = ClockSampler(local_rank).__enter__()  # sampled from warm-up through the last leg
+    time.sleep(0.2)
+    for _ in range(args.warmup):
+        call()
+    if sdpa.get_last_device_error() != sdpa.SDPA_OK:
+        raise SystemExit("device error during warm-up")
+
+    # ---- device-timed region: K steps (one launch each), L2 flushed before each (flush not timed)
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    per_launch = timed_launches(call, args.steps, flush, stream)
+    t_wall1 = time.time()
+    barrier()
+    local_t = float(per_launch.sum())
+    t_max, units = aggregate(local_t, wh.flops() * args.steps)
+    value = units / t_max / 1e12
+    if sdpa.get_last_device_error() != sdpa.SDPA_OK:
+        raise SystemExit("device error in the timed region")
+    t_dom = float(per_launch.mean())
+    roof = tensor_roofline(kernel_name(wh) + " (%s)" % wh.name, wh.flops(), wh.bytes(), t_dom, peaks, peak_kind,
+                           profiled_traffic("prefill_%s_dram.txt" % wh.name, PREFILL_SOURCES),
+                           "profiles/prefill_%s_dram.txt" % wh.name)
+    roof["per_launch_ms"] = round(t_dom * 1e3, 4)
+    roof["per_launch_ms_min"] = round(float(per_launch.min()) * 1e3, 4)
+
+    # ---- end to end through the public API
+    e_local, h2d, d2h = run_e2e(sdpa, wh, inp, stream, args.steps)
+    e_max, e_units = aggregate(e_local, wh.flops() * args.steps)
+    e2e = {"value": round(e_units / e_max / 1e12, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h,
+           "schedule": "steps pipelined: step i+1's inputs copied in and step i-1's outputs copied out "
+                       "(pinned host memory, own streams) while step i computes"}
+    del inp
+
+    # ---- sub-benchmarks: the other prefill workloads, backward, decode (each its own timed loop)
+    legs = {}
+    if not args.skip_legs:
+        for name in args.legs.split(","):
+            if name and name != args.workload:
+                legs[name] = run_prefill_leg(args, sdpa, name, dev, stream, flush, peaks, peak_kind, clocks)
+    backward = {}
+    if not args.skip_backward:
+        for name in filter(None, args.backward_legs.split(",")):
+            backward[name] = run_backward(args, sdpa, si, W, name, dev, stream, flush, peaks, peak_kind, clocks)
+    decode = None if args.skip_decode else run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind,
+                                                      clocks)
+    decode_gqa = (None if args.skip_decode else
+                  run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, clocks, grouped=True))
+    clocks.__exit__(None, None, None)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t_max / args.steps * 1e3, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64/Box-Muller, bf16 RNE)",
+        "config": {"workload": DESCRIBE[wh.name], "global_batch": wh.batch * world, "seq_len": wh.n_q,
+                   "heads": wh.heads, "head_dim": wh.d,
+                   "parallelism": "replicas x%d (independent heads, no collective)" % world,
+                   "l2": "flushed before every timed launch (256 MiB write, not timed); inputs also exceed L2"},
+        "roofline": roof,
+        "cost_model": cost_model(wh.flops(), wh.bytes(), t_dom, peaks, standard_bytes(wh)),
+        "gpu_launches": args.steps,
+        "e2e": e2e,
+        "clocks": clocks.summary(t_wall0, t_wall1),
+        "clocks_all_legs": clocks.summary(t_wall0, time.time()),
+    }
+    if legs:
+        line["prefill_legs"] = legs
+    if backward:
+        line["backward"] = backward
+    if decode is not None:
+        line["decode"] = decode
+    if decode_gqa is not None:
+        line["decode_gqa"] = decode_gqa
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        rate, cores, desc, secs = oracle_rate([wh], args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(rate, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": round(secs, 2)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 # --------------------------------------------------------------------------------------------- reference arm
@@ -524,25 +604,23 @@ def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
         return
-    from seeded_inputs import workloads as W
-    import oracle
-    works = [W.CFG2, W.CFG2C]
+    wh = workload(args.workload)
     for _ in range(args.warmup):
-        oracle_rate(works, 0.2)
+        oracle_rate([wh], 0.2)
     rates, secs = [], 0.0
     desc, cores = "", 1
     for _ in range(args.steps):
-        rate, cores, desc, t = oracle_rate(works, args.cpu_seconds / max(args.steps, 1))
+        rate, cores, desc, t = oracle_rate([wh], args.cpu_seconds / max(args.steps, 1))
         rates.append(rate)
         secs += t
     value = float(np.mean(rates))
-    line = {"impl": "reference", "metric": "attention fwd TFLOP/s (prefill) & decode HBM GB/s, as % of B200 roofline",
+    line = {"impl": "reference", "metric": METRIC,
             "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(secs / args.steps * 1e3, 2), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded SplitMix64/Box-Muller, bf16 RNE)",
-            "config": {"workload": "cfg2: prefill bf16 batch 4 x 16 heads, n_q = n_kv = 2048, d_k = d_v = 64, "
-                                   "scale 1/8, non-causal + causal per step (bounded row sample per step)",
-                       "global_batch": 4, "seq_len": 2048, "parallelism": "host cores"},
+            "config": {"workload": DESCRIBE[wh.name] + " (bounded row sample per step)",
+                       "global_batch": wh.batch, "seq_len": wh.n_q, "heads": wh.heads, "head_dim": wh.d,
+                       "parallelism": "host cores"},
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -555,13 +633,22 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="cfg2", choices=["cfg2", "cfg3", "cfg4", "cfg3w"])
+    ap.add_argument("--workload", default="cfg4", choices=PREFILL_WORKLOADS, help="headline prefill workload")
+    ap.add_argument("--leg-seconds", type=float, default=0.1,
+                    help="device time each sub-benchmark's timed loop fills (at least --steps launches)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
+    ap.add_argument("--legs", default="cfg2,cfg2c,cfg3,cfg3w,cfg4",
+                    help="prefill sub-benchmarks (comma list; the headline workload is skipped)")
+    ap.add_argument("--backward-legs", default="cfg2,cfg2c,cfg3", help="backward sub-benchmarks (comma list)")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-legs", action="store_true", help="no prefill sub-benchmarks")
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=64, help="sequences in the decode workload (default 64)")
     args = ap.parse_args(argv)
+    for name in filter(None, args.legs.split(",") + args.backward_legs.split(",")):
+        if name not in PREFILL_WORKLOADS:
+            raise SystemExit("unknown workload %r (choose from %s)" % (name, ", ".join(PREFILL_WORKLOADS)))
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

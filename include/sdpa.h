@@ -57,7 +57,10 @@ typedef enum {
   SDPA_ERR_WORKSPACE = 4,       /* workspace missing or too small */
   SDPA_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed */
   SDPA_ERR_DEVICE_TIMEOUT = 6,  /* a kernel pipeline wait gave up (device error word) */
-  SDPA_ERR_DEVICE_BAD_LENGTH = 7 /* a decode length was outside [1, n_kv_cap] (device error word) */
+  SDPA_ERR_DEVICE_BAD_LENGTH = 7, /* a decode length was outside [1, n_kv_cap] (device error word) */
+  SDPA_ERR_DEVICE_CHECK = 8     /* debug builds (-DSDPA_DEBUG=1) only: a device-side consistency check
+                                   failed -- a pipeline barrier ended a kernel with a phase count its
+                                   users did not account for, or TMEM was not allocated at column 0 */
 } sdpa_status;
 
 /*

@@ -58,6 +58,7 @@ SDPA_ERR_WORKSPACE = 4
 SDPA_ERR_CUDA = 5
 SDPA_ERR_DEVICE_TIMEOUT = 6
 SDPA_ERR_DEVICE_BAD_LENGTH = 7
+SDPA_ERR_DEVICE_CHECK = 8
 
 
 class SdpaError(RuntimeError):

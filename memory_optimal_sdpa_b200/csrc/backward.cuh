@@ -227,7 +227,9 @@ __global__ void __launch_bounds__(384, 1)
   bool timed_out = false;
   static_assert(C::EW_REGS * 256 + C::CONTROL_REGS * 128 <= 168 * 384, "register split exceeds the launch");
 
-  if (warp >= 8) {
+  const bool tmem_bad = tmem_alloc_bad(tmem);  // debug builds only
+  if (tmem_bad) {
+  } else if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONTROL_REGS));
     if (warp == C::LOAD_WARP) {
       // ------------------------------------------------------------ TMA producer
@@ -508,7 +510,9 @@ __global__ void __launch_bounds__(384, 1)
   bool timed_out = false;
   static_assert(C::EW_REGS * 256 + C::CONTROL_REGS * 128 <= 168 * 384, "register split exceeds the launch");
 
-  if (warp >= 8) {
+  const bool tmem_bad = tmem_alloc_bad(tmem);  // debug builds only
+  if (tmem_bad) {
+  } else if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONTROL_REGS));
     if (warp == C::LOAD_WARP) {
       // ------------------------------------------------------------ TMA producer

@@ -142,8 +142,10 @@ __global__ void __launch_bounds__(192, GqaCfg<NQ>::MIN_BLOCKS)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   bool timed_out = false;
+  const bool tmem_bad = tmem_alloc_bad(tmem);  // debug builds only
 
-  if (warp == 0) {
+  if (tmem_bad) {
+  } else if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);

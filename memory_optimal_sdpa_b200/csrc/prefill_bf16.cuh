@@ -61,7 +61,8 @@ struct PrefillCfg {
   // q_full, full[NSLOT], empty[NSLOT], s_full[2], s_free[2], p_full[2], pv_done[2], o_full[2], drain[2], turn[8],
   // q_free, o_free[2]
   static constexpr int NBAR = 1 + 2 * NSLOT + 2 * 6 + 8 + 3;
-  static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;  // + tmem slot, abort flag, align slack
+  // + tmem slot, abort flag, eight debug counters, align slack
+  static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 48 + 1024;
   static constexpr int THREADS = 384;
   static constexpr int SOFTMAX_REGS = 216;
   static constexpr int CONTROL_REGS = 72;
@@ -81,10 +82,33 @@ __device__ int g_sdpa_error;  // first device-side error since the last read (0 
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_sdpa_error, 0, code); }
 
+// Debug builds (-DSDPA_DEBUG=1) add device-side consistency checks, the stand-in for a race
+// checker on this hardware; a failed check records SDPA_ERR_DEVICE_CHECK (8).  Every tensor-core
+// kernel here runs one CTA per SM and allocates TMEM from column 0, so its allocation must come
+// back at lane 0, column 0; if it does not, the CTA does no work.
+#ifndef SDPA_DEBUG
+#define SDPA_DEBUG 0
+#endif
+__device__ __forceinline__ bool tmem_alloc_bad(uint32_t tmem) {
+#if SDPA_DEBUG
+  if (tmem != 0u) {
+    if (threadIdx.x == 0) record_error(8 /* SDPA_ERR_DEVICE_CHECK */);
+    return true;
+  }
+#endif
+  (void)tmem;
+  return false;
+}
+
 struct PrefillParams {
   __nv_bfloat16* O;
   float* LSE;
   int n_q, n_kv, bh_count, n_pairs;
+  // Units are numbered group of heads by group of heads: within a group of `heads_per_group`
+  // (batch, head) slices (the last group may hold fewer), heaviest query-tile pair first and
+  // the group's heads side by side.  CTAs running at the same time then stream the keys and
+  // values of few heads, which stay in L2 for all of them.
+  int heads_per_group;
   float scale_log2;  // |scale| * log2(e), >= 0
   // scale < 0: the S product is issued with A negated (S = -Q K^T), so the kernel always
   // works with a non-negative factor |scale| (the instruction descriptor's negate-A bit).
@@ -109,6 +133,14 @@ __host__ __device__ inline void prefill_kv_range(int r0, int n_q, int n_kv, int 
   *first = (int)(lo / 128);
   *count = (int)(hi / 128) - *first + 1;
 }
+
+// Heads per unit group (see PrefillParams::heads_per_group).  Full attention: every unit weighs
+// the same, so one head at a time (the CTAs of a round share one or two heads' keys and values).
+// Causal or windowed: unit weights fall with the pair index, and only the order "heaviest pair
+// of every head first" lets the alternating deal balance the CTAs (simulated max/mean load on a
+// 1 x 32 x 8192 causal call: 1.02 with all heads in one group, 1.15-1.47 with groups of 1-16
+// heads), so all heads form one group and keys are re-read from DRAM instead.
+__host__ __device__ inline int prefill_heads_per_group(int mask, int bh_count) { return mask == 0 ? 1 : bh_count; }
 
 #ifndef SDPA_SM_INTPACK
 #define SDPA_SM_INTPACK 0
@@ -199,6 +231,10 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* o_free = q_free + 1;   // [query tile]: the epilogue has read O_x
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  // debug builds: final counters of each role, for the barrier-phase check at teardown
+  // [0] units loaded, [1] ring indices loaded, [2 + x] rounds of tile x, [4 + x] units with rounds
+  // of tile x (softmax x), [6 + x] units seen by issuer x
+  int* dbg = (int*)(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -219,8 +255,13 @@ __global__ void __launch_bounds__(384, 1)
   };
   auto unit_at = [&](int u) {
     Unit g;
-    g.bh = u % p.bh_count;
-    const int pair = p.n_pairs - 1 - u / p.bh_count;
+    const int per_group = p.heads_per_group * p.n_pairs;  // units of a full group
+    const int grp = u / per_group;
+    const int r = u - grp * per_group;
+    const int h0 = grp * p.heads_per_group;
+    const int hg = (p.bh_count - h0 < p.heads_per_group) ? p.bh_count - h0 : p.heads_per_group;
+    g.bh = h0 + r % hg;
+    const int pair = p.n_pairs - 1 - r / hg;
     g.r0a = pair * 256;
     g.r0b = g.r0a + 128;
     prefill_kv_range(g.r0a, p.n_q, p.n_kv, win_left, win_right, &g.fa, &g.ta);  // first key tile, count
@@ -265,8 +306,10 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
   bool timed_out = false;
   static_assert(C::SOFTMAX_REGS * 256 + C::CONTROL_REGS * 128 <= 168 * 384, "register split exceeds the launch");
+  const bool tmem_bad = tmem_alloc_bad(tmem);
 
-  if (warp >= 8) {
+  if (tmem_bad) {
+  } else if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONTROL_REGS));
     if (warp == C::LOAD_WARP) {
       // ------------------------------------------------------------ TMA producer
@@ -303,6 +346,7 @@ __global__ void __launch_bounds__(384, 1)
           if (!ok) break;
           ring += 2 * g.TL;
         }
+        if (SDPA_DEBUG) dbg[0] = nu, dbg[1] = ring;
         if (*abort_flag) {  // let the copies already in flight land before the CTA exits
           if (nu > 0) mbar_wait_drain(q_full, (uint32_t)(nu - 1) & 1u);
           for (int gi = (issued > C::NSLOT ? issued - C::NSLOT : 0); gi < issued; ++gi)
@@ -406,6 +450,7 @@ __global__ void __launch_bounds__(384, 1)
           rx += tx;
           if (tx > 0) ++ox;
         }
+        if (SDPA_DEBUG) dbg[6 + x] = nu;
         // Every MMA and every commit issued above has landed before TMEM is released
         // and before the CTA's shared memory (which the commits arrive on) goes away.
         tc_commit(&drain[x]);
@@ -582,11 +627,31 @@ __global__ void __launch_bounds__(384, 1)
       R += g.T;
       if (tiles > 0) ++ox;
     }
+    if (SDPA_DEBUG && t == 0) dbg[2 + x] = rx, dbg[4 + x] = ox;
   }
 
   if (timed_out) record_error(6 /* SDPA_ERR_DEVICE_TIMEOUT */);
   tc_fence_before_sync();
   __syncthreads();
+#if SDPA_DEBUG
+  // Every barrier has completed exactly as many phases (mod 2) as its users counted: an arrive
+  // too many or too few anywhere in the pipeline shows up here.
+  if (threadIdx.x == 0 && !tmem_bad && !*abort_flag) {
+    bool good = mbar_phase_is(q_full, dbg[0]) && mbar_phase_is(q_free, dbg[0]) && dbg[6] == dbg[0] &&
+                dbg[7] == dbg[0];
+    for (int s = 0; s < C::NSLOT; ++s) {
+      const int n = dbg[1] > s ? (dbg[1] - s + C::NSLOT - 1) / C::NSLOT : 0;
+      good = good && mbar_phase_is(&full[s], n) && mbar_phase_is(&empty[s], n);
+    }
+    for (int x = 0; x < 2; ++x) {
+      const int rx = dbg[2 + x], ox = dbg[4 + x];
+      good = good && mbar_phase_is(&s_full[x], rx) && mbar_phase_is(&p_full[x], rx) &&
+             mbar_phase_is(&o_full[x], ox) && mbar_phase_is(&o_free[x], ox) && mbar_phase_is(&drain[x], 1);
+      if (C::P_SEPARATE) good = good && mbar_phase_is(&s_free[x], rx) && mbar_phase_is(&pv_done[x], rx);
+    }
+    if (!good) record_error(8 /* SDPA_ERR_DEVICE_CHECK */);
+  }
+#endif
   if (warp == C::MMA_WARP) {
     __syncwarp();
     tc_fence_after_sync();

@@ -121,6 +121,7 @@ int launch_prefill(const void* Q, const void* K, const void* V, void* O, float* 
   // persistent: one CTA per SM (at most one per work unit), each striding over the units
   long long grid = (long long)bh * p.n_pairs;
   if (grid > sm_count()) grid = sm_count();
+  p.heads_per_group = sdpa::prefill_heads_per_group(MASK, bh);
   kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess && debug_on()) {
@@ -581,6 +582,7 @@ extern "C" const char* sdpa_status_string(int status) {
     case SDPA_ERR_CUDA: return "SDPA_ERR_CUDA";
     case SDPA_ERR_DEVICE_TIMEOUT: return "SDPA_ERR_DEVICE_TIMEOUT";
     case SDPA_ERR_DEVICE_BAD_LENGTH: return "SDPA_ERR_DEVICE_BAD_LENGTH";
+    case SDPA_ERR_DEVICE_CHECK: return "SDPA_ERR_DEVICE_CHECK";
     default: return "SDPA_UNKNOWN_STATUS";
   }
 }

@@ -50,6 +50,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking: has the phase of `bar` with the given parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// True when the number of completed phases of `bar` has the parity of n (phase n still open).
+__device__ __forceinline__ bool mbar_phase_is(uint64_t* bar, int n) { return !mbar_test_wait(bar, (uint32_t)n & 1u); }
+
 // Wait for the phase of `bar` with the given parity to complete.  Gives up when
 // *abort is set by another thread, or after SDPA_WAIT_BUDGET_NS, in which case it
 // sets *abort itself and returns false (timed_out = true).  Never traps.

@@ -173,7 +173,7 @@ def test_bwd_workspace_and_errors(sdpa):
 
 def test_status_strings(sdpa):
     names = ["SDPA_OK", "SDPA_ERR_INVALID_ARG", "SDPA_ERR_UNSUPPORTED", "SDPA_ERR_MISALIGNED", "SDPA_ERR_WORKSPACE",
-             "SDPA_ERR_CUDA", "SDPA_ERR_DEVICE_TIMEOUT", "SDPA_ERR_DEVICE_BAD_LENGTH"]
+             "SDPA_ERR_CUDA", "SDPA_ERR_DEVICE_TIMEOUT", "SDPA_ERR_DEVICE_BAD_LENGTH", "SDPA_ERR_DEVICE_CHECK"]
     for code, name in enumerate(names):
         assert sdpa.status_string(code) == name
         assert getattr(sdpa, name) == code

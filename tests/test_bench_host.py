@@ -117,9 +117,31 @@ def test_reference_arm_prints_one_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 3
     assert d["value"] > 0 and d["higher_is_better"] is True and d["unit"] == "TFLOP/s"
-    assert d["config"]["workload"].startswith("cfg2")
+    assert d["config"]["workload"].startswith("cfg4")  # the same workload as the headline of our arm
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_roofline_reports_both_denominators():
+    # achieved = algorithmic FLOPs / mean launch time, against the measured burst peak and the spec figure
+    import bench
+    r = bench.tensor_roofline("k", 2e12, 1e9, 0.002, {"bf16_tflops": 1600.0}, "measured", 3e9, "p.txt")
+    assert r["achieved"] == 1000.0 and r["unit"] == "TFLOP/s" and r["bound"] == "tensor"
+    assert r["frac"] == 0.625 and r["peak"] == 1600.0
+    assert r["spec_peak"] == 2250.0 and abs(r["spec_frac"] - 1000.0 / 2250.0) < 1e-4
+    assert r["traffic"] == 3e9 and r["traffic_over_algorithmic_bytes"] == 3.0
+    h = bench.hbm_roofline("d", 6e9, 0.001, {"hbm_gbs": 6000.0}, "measured", None)
+    assert h["achieved"] == 6000.0 and h["frac"] == 1.0 and h["spec_frac"] == 0.75 and h["traffic"] is None
+
+
+def test_every_prefill_workload_is_described_and_defined():
+    import bench
+    from seeded_inputs import workloads as W
+    for name in bench.PREFILL_WORKLOADS:
+        w = bench.workload(name)
+        assert w.name == name and bench.DESCRIBE[name].startswith(name + ":")
+        assert bench.kernel_name(w).startswith("sdpa_fwd_bf16_kernel<%d," % w.d)
+    assert bench.kernel_name(W.CFG3W).endswith(",2>") and bench.kernel_name(W.CFG3).endswith(",1>")
