@@ -72,7 +72,9 @@ typedef enum {
  * causal: 0 or 1.  scale: any finite value (else SDPA_ERR_INVALID_ARG).  A negative
  * scale is applied by negating Q inside the S = Q K^T product (the instruction's
  * negate-A bit), so the online softmax always works with |scale|; scale == 0 gives every
- * visible key weight 1 / (number of visible keys) and LSE = ln(number of visible keys).
+ * visible key weight 1 / (number of visible keys) and LSE = ln(number of visible keys)
+ * (computed with the factor 2^-126 in place of 0, which leaves every weight exactly 1 in
+ * fp32 for scores below 2^100 in magnitude and keeps masked entries at weight 0).
  * Every pointer 16-byte aligned (TMA), else SDPA_ERR_MISALIGNED.
  * Arithmetic: S = Q K^T and O += P V on the tensor cores with fp32
  * accumulation; softmax in fp32 with P rounded to bf16; O rounded to bf16

@@ -109,7 +109,7 @@ struct PrefillParams {
   // the group's heads side by side.  CTAs running at the same time then stream the keys and
   // values of few heads, which stay in L2 for all of them.
   int heads_per_group;
-  float scale_log2;  // |scale| * log2(e), >= 0
+  float scale_log2;  // |scale| * log2(e), > 0 (2^-126 stands for scale = 0)
   // scale < 0: the S product is issued with A negated (S = -Q K^T), so the kernel always
   // works with a non-negative factor |scale| (the instruction descriptor's negate-A bit).
   int negate_s;
@@ -166,8 +166,7 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
 
 // Exponentials of one 128-score row: p = 2^(s*c2 - m), bf16 pairs into pk, returns sum p.
 // EVERY > 0: every EVERY-th pair on the FMA pipe (finite scores only).
-// MASKED: entries set to -inf give p = 0 whatever c2 is (with c2 = 0, -inf * c2 would be NaN).
-template <int EVERY, bool MASKED = false>
+template <int EVERY>
 __device__ __forceinline__ float softmax_exp_row(const uint32_t (&s)[128], float c2, float m_use, uint32_t (&pk)[64]) {
   using namespace sm100;
   const float2 cc = make_float2(c2, c2), nm = make_float2(-m_use, -m_use);
@@ -181,10 +180,6 @@ __device__ __forceinline__ float softmax_exp_row(const uint32_t (&s)[128], float
     } else {
       e.x = ex2_approx(xv.x);
       e.y = ex2_approx(xv.y);
-    }
-    if (MASKED) {
-      if (s[2 * i] == 0xff800000u) e.x = 0.f;
-      if (s[2 * i + 1] == 0xff800000u) e.y = 0.f;
     }
     if (i & 1)
       acc1 = fadd2(acc1, e);
@@ -572,7 +567,7 @@ __global__ void __launch_bounds__(384, 1)
         if (SDPA_SM_TURN && !(ok = wait_warp(my_turn, R + j))) break;  // this warp's turn on the exponentials
         const float m_use = (m_u == NEG_INF) ? 0.f : m_u;
         uint32_t pk[64];
-        l += masked ? softmax_exp_row<0, true>(s, c2, m_use, pk) : softmax_exp_row<C::POLY_EVERY>(s, c2, m_use, pk);
+        l += masked ? softmax_exp_row<0>(s, c2, m_use, pk) : softmax_exp_row<C::POLY_EVERY>(s, c2, m_use, pk);
         if (SDPA_SM_TURN) mbar_arrive(their_turn);  // hand the exponentials over
         if (C::P_SEPARATE && rx + j > 0 && !pv_waited) {  // the last P_x V (this unit's or the previous one's) reads P_x
           if (!(ok = wait_warp(&pv_done[x], rx + j - 1))) break;

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cfloat>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -114,7 +115,10 @@ int launch_prefill(const void* Q, const void* K, const void* V, void* O, float* 
   p.n_kv = n_kv;
   p.bh_count = bh;
   p.n_pairs = (n_q + 255) / 256;
-  p.scale_log2 = std::fabs(scale) * 1.4426950408889634f;
+  // scale = 0 runs with the smallest normal float as the factor: every finite score s then gets
+  // 2^(s * 2^-126 - m) = 1 exactly in fp32 (|s| < 2^100), the weights are uniform as the definition
+  // says, and masked entries (-inf) still give 0, where a factor of exactly 0 would give -inf * 0 = NaN.
+  p.scale_log2 = scale == 0.f ? FLT_MIN : std::fabs(scale) * 1.4426950408889634f;
   p.negate_s = scale < 0.f ? 1 : 0;
   p.win_left = win_left;
   p.win_right = win_right;
