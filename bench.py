@@ -557,10 +557,11 @@ def run_ours(args):
     if not args.skip_backward:
         for name in filter(None, args.backward_legs.split(",")):
             backward[name] = run_backward(args, sdpa, si, W, name, dev, stream, flush, peaks, peak_kind, clocks)
-    decode = None if args.skip_decode else run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind,
-                                                      clocks)
-    decode_gqa = (None if args.skip_decode else
-                  run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, clocks, grouped=True))
+    dlegs = [] if args.skip_decode else args.decode_legs.split(",")
+    decode = (run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, clocks) if "cfg5" in dlegs
+              else None)
+    decode_gqa = (run_decode(args, sdpa, si, W, dev, stream, flush, peaks, peak_kind, clocks, grouped=True)
+                  if "cfg5g" in dlegs else None)
     clocks.__exit__(None, None, None)
 
     line = {
@@ -640,6 +641,7 @@ def main(argv=None):
     ap.add_argument("--legs", default="cfg2,cfg2c,cfg3,cfg3w,cfg4",
                     help="prefill sub-benchmarks (comma list; the headline workload is skipped)")
     ap.add_argument("--backward-legs", default="cfg2,cfg2c,cfg3", help="backward sub-benchmarks (comma list)")
+    ap.add_argument("--decode-legs", default="cfg5,cfg5g", help="decode sub-benchmarks (comma list of cfg5, cfg5g)")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-legs", action="store_true", help="no prefill sub-benchmarks")
     ap.add_argument("--skip-decode", action="store_true")
@@ -649,6 +651,9 @@ def main(argv=None):
     for name in filter(None, args.legs.split(",") + args.backward_legs.split(",")):
         if name not in PREFILL_WORKLOADS:
             raise SystemExit("unknown workload %r (choose from %s)" % (name, ", ".join(PREFILL_WORKLOADS)))
+    for name in filter(None, args.decode_legs.split(",")):
+        if name not in ("cfg5", "cfg5g"):
+            raise SystemExit("unknown decode workload %r (choose from cfg5, cfg5g)" % name)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
