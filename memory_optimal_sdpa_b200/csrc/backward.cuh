@@ -65,8 +65,8 @@ struct BwdCfg {
   static constexpr int FIX_OFF = 0;                // the CTA's fixed pair: (K, V) or (Q, dO)
   static constexpr int ST_OFF = 2 * TILE_BYTES;    // streamed stages: (Q, dO, vectors) or (K, V)
   static constexpr int BAR_OFF = ST_OFF + NSTAGE * STAGE_BYTES;
-  // fix_full, full[NSTAGE], empty[NSTAGE], s_full[2], p_full[2], grad_done[2], o_full, drain[2]
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 9;
+  // fix_full, full[NSTAGE], empty[NSTAGE], s_full[2], p_full[2], grad_done[2], o_full, drain[2], fix_tmem
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 10;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;
   static constexpr int THREADS = 384;
   static constexpr int EW_REGS = 192;  // 192 x 256 + 120 x 128 = 168 x 384: no spills in the control warps
@@ -79,6 +79,13 @@ struct BwdCfg {
   static constexpr uint32_t COL_B = 256 + D;  // accumulator: dK (dkdv)
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr bool TWO_ISSUERS = D >= SDPA_BWD_TWO_ISSUERS_MIN_D;
+  // d = 64: the CTA's fixed pair (K, V in dkdv; Q, dO in dq), the A operands of the S and dP
+  // products, is copied once into TMEM columns [384, 448), so those products read only their B
+  // operand from shared memory (with both operands there, an N = 64 product moves 6 KB of shared
+  // memory per 32 clocks of math, about the SM's shared-memory bandwidth).  At d = 128 the S, dP
+  // and gradient accumulators fill all 512 columns.
+  static constexpr bool FIX_IN_TMEM = (D == 64);
+  static constexpr uint32_t COL_FIX = 384;
 };
 
 // Programmatic dependent launch.  launch_dependents: the next kernel on the stream, if launched
@@ -181,6 +188,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* grad_done = p_full + 2;      // [half]: the gradient products reading half h completed
   uint64_t* o_full = grad_done + 2;
   uint64_t* drain = o_full + 1;          // [issuer]
+  uint64_t* fix_tmem = drain + 2;        // d = 64: the fixed pair has been copied into TMEM
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -213,6 +221,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(o_full, 1);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    mbar_init(fix_tmem, 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -285,8 +294,13 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t o = (uint64_t)((((kk >> 2) * C::BLOCK_BYTES) + (kk & 3) * 32) >> 4);
-            mma_ss(tmem + C::COL_S + 64 * h, dK + o, dQk + o, idS, kk > 0 ? 1u : 0u);
-            mma_ss(tmem + C::COL_DP + 64 * h, dV + o, dOk + o, idS, kk > 0 ? 1u : 0u);
+            if (C::FIX_IN_TMEM) {  // K, V from TMEM: 16 keys' columns are 8 TMEM columns of bf16 pairs
+              mma_ts(tmem + C::COL_S + 64 * h, tmem + C::COL_FIX + kk * 8, dQk + o, idS, kk > 0 ? 1u : 0u);
+              mma_ts(tmem + C::COL_DP + 64 * h, tmem + C::COL_FIX + 32 + kk * 8, dOk + o, idS, kk > 0 ? 1u : 0u);
+            } else {
+              mma_ss(tmem + C::COL_S + 64 * h, dK + o, dQk + o, idS, kk > 0 ? 1u : 0u);
+              mma_ss(tmem + C::COL_DP + 64 * h, dV + o, dOk + o, idS, kk > 0 ? 1u : 0u);
+            }
           }
           tc_commit(&s_full[h]);
         };
@@ -307,7 +321,7 @@ __global__ void __launch_bounds__(384, 1)
         // warpgroup's elementwise pass overlaps the other's and the tensor core's products.
         bool ok = true;
         if (!C::TWO_ISSUERS) {
-          ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0);
+          ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0) && (!C::FIX_IN_TMEM || wait_bar(fix_tmem, 0));
           if (ok) {
             issue_sdp(0, 0);
             issue_sdp(0, 1);
@@ -325,7 +339,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           if (ok) tc_commit(o_full);
         } else if (role == 0) {  // S / dP: half h of tile t once the gradient products of half h of t - 1 are done
-          ok = wait_bar(fix_full, 0);
+          ok = wait_bar(fix_full, 0) && (!C::FIX_IN_TMEM || wait_bar(fix_tmem, 0));
           for (int t = 0; ok && t < NT; ++t)
             for (int h = 0; ok && h < 2; ++h) {
               if (h == 0 && !(ok = wait_bar(&full[t % C::NSTAGE], t / C::NSTAGE))) break;
@@ -359,6 +373,22 @@ __global__ void __launch_bounds__(384, 1)
       const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
       return __all_sync(0xffffffffu, r);
     };
+    if (C::FIX_IN_TMEM && NT > 0 && (ok = wait_warp(fix_full, 0))) {
+      // row `row` of fixed tile w into this warp's TMEM lanes, 32 columns of bf16 pairs: the
+      // 128-byte rows sit in 1 KB atoms of eight, their 16-byte chunks permuted by the
+      // 128-byte swizzle (chunk c of row r at position c ^ (r % 8))
+      const uint8_t* rp = sFix + w * C::TILE_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+      uint32_t v[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 q4 = *reinterpret_cast<const uint4*>(rp + ((c ^ (row & 7)) << 4));
+        v[4 * c] = q4.x, v[4 * c + 1] = q4.y, v[4 * c + 2] = q4.z, v[4 * c + 3] = q4.w;
+      }
+      tmem_st_32x32b_x32(tmem + C::COL_FIX + 32u * (uint32_t)w + lane_base, v);
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(fix_tmem);
+    }
     for (int t = 0; ok && t < NT; ++t) {
       const int st = t % C::NSTAGE;
       const float* vL2 = reinterpret_cast<const float*>(sSt + st * C::STAGE_BYTES + 2 * C::TILE_BYTES);
@@ -465,6 +495,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* grad_done = p_full + 2;      // [half]: the gradient products reading half h completed
   uint64_t* o_full = grad_done + 2;
   uint64_t* drain = o_full + 1;          // [issuer]
+  uint64_t* fix_tmem = drain + 2;        // d = 64: the fixed pair has been copied into TMEM
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -496,6 +527,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(o_full, 1);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    mbar_init(fix_tmem, 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -562,8 +594,13 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t o = (uint64_t)((((kk >> 2) * C::BLOCK_BYTES) + (kk & 3) * 32) >> 4);
-            mma_ss(tmem + C::COL_S + 64 * h, dQk + o, dKk + o, idS, kk > 0 ? 1u : 0u);
-            mma_ss(tmem + C::COL_DP + 64 * h, dOk + o, dVk + o, idS, kk > 0 ? 1u : 0u);
+            if (C::FIX_IN_TMEM) {  // Q, dO from TMEM
+              mma_ts(tmem + C::COL_S + 64 * h, tmem + C::COL_FIX + kk * 8, dKk + o, idS, kk > 0 ? 1u : 0u);
+              mma_ts(tmem + C::COL_DP + 64 * h, tmem + C::COL_FIX + 32 + kk * 8, dVk + o, idS, kk > 0 ? 1u : 0u);
+            } else {
+              mma_ss(tmem + C::COL_S + 64 * h, dQk + o, dKk + o, idS, kk > 0 ? 1u : 0u);
+              mma_ss(tmem + C::COL_DP + 64 * h, dOk + o, dVk + o, idS, kk > 0 ? 1u : 0u);
+            }
           }
           tc_commit(&s_full[h]);
         };
@@ -578,7 +615,7 @@ __global__ void __launch_bounds__(384, 1)
         };
         bool ok = true;
         if (!C::TWO_ISSUERS) {
-          ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0);
+          ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0) && (!C::FIX_IN_TMEM || wait_bar(fix_tmem, 0));
           if (ok) {
             issue_sdp(0, 0);
             issue_sdp(0, 1);
@@ -596,7 +633,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           if (ok) tc_commit(o_full);
         } else if (role == 0) {
-          ok = wait_bar(fix_full, 0);
+          ok = wait_bar(fix_full, 0) && (!C::FIX_IN_TMEM || wait_bar(fix_tmem, 0));
           for (int j = 0; ok && j < T; ++j)
             for (int h = 0; ok && h < 2; ++h) {
               if (h == 0 && !(ok = wait_bar(&full[j % C::NSTAGE], j / C::NSTAGE))) break;
@@ -634,6 +671,20 @@ __global__ void __launch_bounds__(384, 1)
       const bool r = mbar_wait_bounded(bar, (uint32_t)phase & 1u, abort_flag, &timed_out);
       return __all_sync(0xffffffffu, r);
     };
+    if (C::FIX_IN_TMEM && T > 0 && (ok = wait_warp(fix_full, 0))) {
+      // row `row` of fixed tile w (Q or dO) into this warp's TMEM lanes, as in the dK/dV kernel
+      const uint8_t* rp = sFix + w * C::TILE_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+      uint32_t v[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 q4 = *reinterpret_cast<const uint4*>(rp + ((c ^ (row & 7)) << 4));
+        v[4 * c] = q4.x, v[4 * c + 1] = q4.y, v[4 * c + 2] = q4.z, v[4 * c + 3] = q4.w;
+      }
+      tmem_st_32x32b_x32(tmem + C::COL_FIX + 32u * (uint32_t)w + lane_base, v);
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(fix_tmem);
+    }
     for (int j = 0; ok && j < T; ++j) {
       if (!(ok = wait_warp(&s_full[w], j))) break;
       tc_fence_after_sync();
