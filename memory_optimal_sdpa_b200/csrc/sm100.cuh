@@ -85,6 +85,35 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Monotonic counters in shared memory: red.release / ld.acquire at CTA scope.
+__device__ __forceinline__ void red_release_add(uint32_t* word, uint32_t v) {
+  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(word)), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* word) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(word)) : "memory");
+  return v;
+}
+// Wait until *counter >= target.  Unlike a phase-parity wait, a count cannot be mistaken for an
+// earlier or later phase however far the waiter is ahead or behind.  Bounded as mbar_wait_bounded.
+__device__ __forceinline__ bool count_wait_bounded(const uint32_t* counter, uint32_t target, volatile int* abort,
+                                                   bool* timed_out) {
+  if (ld_acquire(counter) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(32);
+    if (ld_acquire(counter) >= target) return true;
+    if ((it & 15u) == 0) {
+      if (abort && *abort) return false;
+      if (globaltimer_ns() - t0 > SDPA_WAIT_BUDGET_NS) {
+        if (abort) *abort = 1;
+        *timed_out = true;
+        return false;
+      }
+    }
+  }
+}
+
 // Cleanup wait after an abort: bounded by time only.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
