@@ -52,6 +52,9 @@
 #ifndef SDPA_EXP2_POLY_EVERY_D64
 #define SDPA_EXP2_POLY_EVERY_D64 8  // every 8th column pair of an unmasked tile on the FMA pipe at d = 64
 #endif
+#ifndef SDPA_EXP2_POLY_EVERY_D128
+#define SDPA_EXP2_POLY_EVERY_D128 0  // the same at d = 128 (0: all exponentials on the MUFU unit)
+#endif
 
 namespace sdpa {
 
@@ -81,7 +84,7 @@ struct PrefillCfg {
   // the next S no longer waits for P_x V.
   static constexpr bool SHARED_S = (D == 128) && SDPA_SHARED_S_D128;
   static constexpr bool P_SEPARATE = (D == 64) || SHARED_S;
-  static constexpr int POLY_EVERY = (D == 64) ? SDPA_EXP2_POLY_EVERY_D64 : 0;  // FMA-pipe exponentials
+  static constexpr int POLY_EVERY = (D == 64) ? SDPA_EXP2_POLY_EVERY_D64 : SDPA_EXP2_POLY_EVERY_D128;  // FMA-pipe exps
   __host__ __device__ static constexpr uint32_t col_s(int x) { return SHARED_S ? 0u : (uint32_t)x * 128u; }
   __host__ __device__ static constexpr uint32_t col_p(int x) {
     return D == 64 ? 256u + (uint32_t)x * 64u : (SHARED_S ? 128u + (uint32_t)x * 64u : col_s(x));
