@@ -38,6 +38,10 @@
 #define SDPA_BWD_TWO_ISSUERS_MIN_D 128
 #endif
 
+#ifndef SDPA_BWD_DS_SEPARATE_D64
+#define SDPA_BWD_DS_SEPARATE_D64 0  // measured: d = 64 backward 427 -> 414 TF/s with it, d = 128 709 -> 716
+#endif
+
 namespace sdpa {
 
 struct BwdParams {
@@ -65,8 +69,9 @@ struct BwdCfg {
   static constexpr int FIX_OFF = 0;                // the CTA's fixed pair: (K, V) or (Q, dO)
   static constexpr int ST_OFF = 2 * TILE_BYTES;    // streamed stages: (Q, dO, vectors) or (K, V)
   static constexpr int BAR_OFF = ST_OFF + NSTAGE * STAGE_BYTES;
-  // fix_full, full[NSTAGE], empty[NSTAGE], s_full[2], p_full[2], grad_done[2], o_full, drain[2], fix_tmem
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 10;
+  // fix_full, full[NSTAGE], empty[NSTAGE], s_full[2], p_full[2], grad_done[2], o_full, drain[2], fix_tmem,
+  // sd_free[2]
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 12;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;
   static constexpr int THREADS = 384;
   static constexpr int EW_REGS = 192;  // 192 x 256 + 120 x 128 = 168 x 384: no spills in the control warps
@@ -86,6 +91,11 @@ struct BwdCfg {
   // and gradient accumulators fill all 512 columns.
   static constexpr bool FIX_IN_TMEM = (D == 64);
   static constexpr uint32_t COL_FIX = 384;
+  // dq kernel: dS in columns of its own (bf16 pairs, 32 per warpgroup) instead of over dP, so
+  // the next key tile's S and dP products need only wait until the elementwise warps have read
+  // S and dP, not until the dQ product has read dS.
+  static constexpr bool DS_SEPARATE = SDPA_BWD_DS_SEPARATE_D64 || D == 128;
+  static constexpr uint32_t COL_DS = FIX_IN_TMEM ? 448 : 384;
 };
 
 // Programmatic dependent launch.  launch_dependents: the next kernel on the stream, if launched
@@ -189,6 +199,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* o_full = grad_done + 2;
   uint64_t* drain = o_full + 1;          // [issuer]
   uint64_t* fix_tmem = drain + 2;        // d = 64: the fixed pair has been copied into TMEM
+  uint64_t* sd_free = fix_tmem + 1;      // [half] (dq): S and dP of half h are in registers
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -222,6 +233,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     mbar_init(fix_tmem, 256);
+    mbar_init(&sd_free[0], 128);
+    mbar_init(&sd_free[1], 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -496,6 +509,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* o_full = grad_done + 2;
   uint64_t* drain = o_full + 1;          // [issuer]
   uint64_t* fix_tmem = drain + 2;        // d = 64: the fixed pair has been copied into TMEM
+  uint64_t* sd_free = fix_tmem + 1;      // [half] (dq): S and dP of half h are in registers
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -528,6 +542,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     mbar_init(fix_tmem, 256);
+    mbar_init(&sd_free[0], 128);
+    mbar_init(&sd_free[1], 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -609,8 +625,10 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4) {
             const int kk = 4 * h + k4;
-            mma_ts(tmem + C::COL_A, tmem + C::COL_DP + bwd_pair_col(kk), dKm + (uint64_t)((kk * 2048) >> 4), idA,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+            // dS pairs: in their own columns (32 per warpgroup) or over dP (bwd_pair_col)
+            const uint32_t a_col = C::DS_SEPARATE ? C::COL_DS + (uint32_t)((kk >> 2) * 32 + (kk & 3) * 8)
+                                                  : C::COL_DP + bwd_pair_col(kk);
+            mma_ts(tmem + C::COL_A, tmem + a_col, dKm + (uint64_t)((kk * 2048) >> 4), idA, (j > 0 || kk > 0) ? 1u : 0u);
           }
         };
         bool ok = true;
@@ -622,10 +640,16 @@ __global__ void __launch_bounds__(384, 1)
           }
           for (int j = 0; ok && j < T; ++j) {
             for (int h = 0; ok && h < 2; ++h) {
+              if (C::DS_SEPARATE && j + 1 < T) {  // next S / dP of half h once S, dP of half h are read
+                if (h == 0 && !(ok = wait_bar(&full[(j + 1) % C::NSTAGE], (j + 1) / C::NSTAGE))) break;
+                if (!(ok = wait_bar(&sd_free[h], j))) break;
+                issue_sdp(j + 1, h);
+              }
               if (!(ok = wait_bar(&p_full[h], j))) break;
               issue_grad(j, h);
+              if (C::DS_SEPARATE) tc_commit(&grad_done[h]);
               if (h == 1) tc_commit(&empty[j % C::NSTAGE]);
-              if (j + 1 < T) {
+              if (!C::DS_SEPARATE && j + 1 < T) {
                 if (h == 0 && !(ok = wait_bar(&full[(j + 1) % C::NSTAGE], (j + 1) / C::NSTAGE))) break;
                 issue_sdp(j + 1, h);
               }
@@ -637,7 +661,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int j = 0; ok && j < T; ++j)
             for (int h = 0; ok && h < 2; ++h) {
               if (h == 0 && !(ok = wait_bar(&full[j % C::NSTAGE], j / C::NSTAGE))) break;
-              if (j > 0 && !(ok = wait_bar(&grad_done[h], j - 1))) break;
+              if (j > 0 && !(ok = wait_bar(C::DS_SEPARATE ? &sd_free[h] : &grad_done[h], j - 1))) break;
               issue_sdp(j, h);
             }
         } else {
@@ -699,6 +723,17 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_ld();
         reg_fence(s);
         reg_fence(dp);
+        if (C::DS_SEPARATE && h == 0) {
+          // the last dQ product reading this warpgroup's dS columns has completed
+          if (j > 0 && !(ok = wait_warp(&grad_done[w], j - 1))) break;
+          tc_fence_after_sync();
+        }
+        if (C::DS_SEPARATE && h == 1) {
+          // this warpgroup's S and dP columns are all in registers: with dS in columns of its own
+          // the tensor core may overwrite them with the next key tile's S and dP
+          tc_fence_before_sync();
+          mbar_arrive(&sd_free[w]);
+        }
         uint32_t pp[16], ps[16];
         const int kc = k0 + 32 * h;
         if (masked)
@@ -707,8 +742,11 @@ __global__ void __launch_bounds__(384, 1)
         else
           bwd_elementwise(s, dp, c2, [&](int) { return l2; }, [&](int) { return dd; }, [&](int) { return true; }, pp,
                           ps);
-        tmem_st_32x32b_x16(tmem + C::COL_DP + (uint32_t)(64 * w + 16 * h) + lane_base, ps);
+        const uint32_t col =
+            C::DS_SEPARATE ? C::COL_DS + (uint32_t)(32 * w + 16 * h) : C::COL_DP + (uint32_t)(64 * w + 16 * h);
+        tmem_st_32x32b_x16(tmem + col + lane_base, ps);
       }
+      if (!ok) break;
       tmem_wait_st();
       tc_fence_before_sync();
       mbar_arrive(&p_full[w]);
