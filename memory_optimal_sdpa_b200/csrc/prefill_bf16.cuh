@@ -167,6 +167,9 @@ __host__ __device__ inline int prefill_heads_per_group(int mask, int bh_count) {
 #ifndef SDPA_SM_TURN_WARP
 #define SDPA_SM_TURN_WARP 1
 #endif
+#ifndef SDPA_SM_TURN_NAMED
+#define SDPA_SM_TURN_NAMED 1  // pass the turn with hardware named barriers (else mbarriers)
+#endif
 
 // Two finite, non-negative floats -> bf16x2 (lo in bits 0..15), rounded to nearest.
 // Default: the packed conversion instruction (measured on B200 at 62 per clock per SM, on a
@@ -515,7 +518,45 @@ __global__ void __launch_bounds__(384, 1)
     // b is tile a's first turn of the next unit.
     uint64_t* my_turn = &turn[SDPA_SM_TURN_WARP ? 4 * x + (warp & 3) : 4 * x];
     uint64_t* their_turn = &turn[SDPA_SM_TURN_WARP ? 4 * (x ^ 1) + (warp & 3) : 4 * (x ^ 1)];
-    if (SDPA_SM_TURN && x == 1) mbar_arrive(their_turn);
+    // SDPA_SM_TURN_NAMED: the turn passes through hardware named barriers instead (ids 1-8, one per
+    // sub-partition and tile, 64 threads: the passing warp's bar.arrive and the taking warp's
+    // bar.sync), whose release takes tens of clocks where an mbarrier wake-up took about 340.  A
+    // named barrier cannot time out, so each warp runs exactly turn_total wait/pass pairs -- one
+    // per round of every unit of this CTA, the same count for both warps of a pair -- even after a
+    // failed wait: it then drops the work but keeps taking and passing its turns until the count is
+    // reached, so its partner is never left at a barrier.  Tile b's very first pass is tile a's
+    // first turn, and b's last pass, which no round would take, is not made.
+    const int turn_mine = 1 + 4 * x + (warp & 3), turn_theirs = 1 + 4 * (x ^ 1) + (warp & 3);
+    int R_turn = 0;  // the current round's turn phase (mbarrier turns)
+    int turn_total = 0, turn_done = 0;
+    if (SDPA_SM_TURN && SDPA_SM_TURN_NAMED)
+      for (int k = 0, u = unit_of(0); u < n_units; u = unit_of(++k)) turn_total += unit_at(u).T;
+    // (bar.sync / bar.arrive are whole-warp instructions: the warp is reconverged first, since the
+    // per-row choice of exponential loop may have split it)
+    auto turn_wait = [&]() -> bool {
+      if (SDPA_SM_TURN_NAMED) {
+        __syncwarp();
+        named_bar_sync(turn_mine, 64);
+        return true;
+      }
+      return wait_warp(my_turn, R_turn);
+    };
+    auto turn_pass = [&]() {
+      if (SDPA_SM_TURN_NAMED) {
+        __syncwarp();
+        if (!(x == 1 && turn_done + 1 == turn_total)) named_bar_arrive(turn_theirs, 64);
+        ++turn_done;
+      } else {
+        mbar_arrive(their_turn);
+      }
+    };
+    if (SDPA_SM_TURN && x == 1) {
+      if (!SDPA_SM_TURN_NAMED) mbar_arrive(their_turn);
+      else if (turn_total > 0) {
+        __syncwarp();
+        named_bar_arrive(turn_theirs, 64);
+      }
+    }
     int rx = 0, R = 0, ox = 0;  // rounds of this tile so far, rounds of both, units with rounds
     for (int k = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++k)) {
       const Unit g = unit_at(u);
@@ -532,10 +573,11 @@ __global__ void __launch_bounds__(384, 1)
       float m_u = NEG_INF;  // running max of scale*log2(e)*s
       float l = 0.f;
       for (int j = 0; ok && j < g.T; ++j) {
+        R_turn = R + j;
         if (j >= tiles) {  // no key tile left for this query tile: only pass the turn
           if (SDPA_SM_TURN) {
-            if (!(ok = wait_warp(my_turn, R + j))) break;
-            mbar_arrive(their_turn);
+            if (!(ok = turn_wait())) break;
+            turn_pass();
           }
           continue;
         }
@@ -603,11 +645,11 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
         }
-        if (SDPA_SM_TURN && !(ok = wait_warp(my_turn, R + j))) break;  // this warp's turn on the exponentials
+        if (SDPA_SM_TURN && !(ok = turn_wait())) break;  // this warp's turn on the exponentials
         const float m_use = (m_u == NEG_INF) ? 0.f : m_u;
         uint32_t pk[64];
         l += masked ? softmax_exp_row<0>(s, c2, m_use, pk) : softmax_exp_row<C::POLY_EVERY>(s, c2, m_use, pk);
-        if (SDPA_SM_TURN) mbar_arrive(their_turn);  // hand the exponentials over
+        if (SDPA_SM_TURN) turn_pass();  // hand the exponentials over
         if (C::P_SEPARATE && rx + j > 0 && !pv_waited) {  // the last P_x V (this unit's or the previous one's) reads P_x
           if (!(ok = wait_warp(&pv_done[x], rx + j - 1))) break;
           tc_fence_after_sync();
@@ -661,6 +703,12 @@ __global__ void __launch_bounds__(384, 1)
       R += g.T;
       if (tiles > 0) ++ox;
     }
+    // After a failed wait: the remaining turns, without the work (named barriers cannot time out)
+    if (SDPA_SM_TURN && SDPA_SM_TURN_NAMED)
+      while (turn_done < turn_total) {
+        turn_wait();
+        turn_pass();
+      }
     if (SDPA_DEBUG && t == 0) dbg[2 + x] = rx, dbg[4 + x] = ox;
   }
 

@@ -281,6 +281,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+// Arrive at a named barrier without waiting (the waiting side uses named_bar_sync).
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 // Barrier that also returns whether `pred` held on any participating thread.
 __device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
   uint32_t r;
