@@ -498,6 +498,14 @@ def test_decode_gqa_multi_tile_splits(sdpa, cuda_device):
     _gqa_medium(sdpa, cuda_device, q, k, v, lens, float(np.float32(1 / math.sqrt(d))), "gqa multi-tile")
 
 
+def test_decode_gqa_zero_scale(sdpa, cuda_device):
+    # scale 0: every query head of a group gets the mean of its sequence's visible value rows
+    B, H_q, H_kv, n_cap, d = 4, 16, 2, 3000, 128
+    lens = np.array([1, 3000, 1500, 129], np.int32)
+    q, k, v = _gqa_inputs(B, H_q, H_kv, n_cap, d, lens, 31)
+    _gqa_medium(sdpa, cuda_device, q, k, v, lens, 0.0, "gqa scale 0")
+
+
 def test_decode_gqa_rescale_inside_a_split(sdpa, cuda_device):
     # Scores that climb by ~12 (log2 units) from one 128-key tile to the next move every
     # head's reference maximum inside a split; a negative scale is accepted here too.
@@ -569,6 +577,26 @@ def test_prefill_f32(sdpa, cuda_device, B, H, n_q, n_kv, dk, dv, causal):
     check_lse(lse.cpu().numpy(), L_ref, 1e-5, "f32")
 
 
+@pytest.mark.parametrize("scale", [0.0, -0.125, -0.0883883461356163])
+@pytest.mark.parametrize("causal", [False, True])
+def test_prefill_f32_zero_and_negative_scale(sdpa, cuda_device, causal, scale):
+    # any finite scale on the CUDA-core path too: 0 gives the mean of the visible rows, a negative
+    # scale flips the logits (rows 0.. of a causal call see 1.. keys).  Scales of the fp32
+    # workload's magnitude: the 1e-5 relative bound holds for logits of that size (at |scale| = 1
+    # the fp32 rounding of the 64-term dot products alone, about |s| 2^-24 sqrt(d), exceeds it).
+    B, H, n_q, n_kv, d = 1, 2, 150, 170, 64
+    q = si.fill_host((B, H, n_q, d), 8, 0, bf16=False)
+    k = si.fill_host((B, H, n_kv, d), 8, 1, bf16=False)
+    v = si.fill_host((B, H, n_kv, d), 8, 2, bf16=False)
+    tq, tk, tv = (W.to_torch(x, cuda_device) for x in (q, k, v))
+    o, lse = sdpa.fwd_f32(tq, tk, tv, causal=causal, scale=scale)
+    assert sdpa.get_last_device_error() == sdpa.SDPA_OK
+    O_ref, L_ref = oracle.sdpa_rows(q, k, v, scale, causal)
+    err = np.abs(o.cpu().numpy().astype(np.float64) - O_ref)
+    assert (err <= 1e-5 * np.abs(O_ref) + 1e-6).all(), "scale %g: max err %.3g" % (scale, err.max())
+    check_lse(lse.cpu().numpy(), L_ref, 1e-5, "f32 scale %g" % scale)
+
+
 def test_cfg1_fp32(sdpa, cuda_device):
     w = W.CFG1
     host = W.prefill_host(w)
@@ -581,8 +609,9 @@ def test_cfg1_fp32(sdpa, cuda_device):
 
 
 # -------------------------------------------------------------------------------------------------- decode
+@pytest.mark.parametrize("scale_kind", ["default", "zero", "negative"])
 @pytest.mark.parametrize("d", [64, 128])
-def test_decode_small_every_pair(sdpa, cuda_device, d):
+def test_decode_small_every_pair(sdpa, cuda_device, d, scale_kind):
     import torch
     B, H, n_cap = 3, 4, 1000
     lens = np.array([1, 1000, 517], np.int32)
@@ -592,13 +621,15 @@ def test_decode_small_every_pair(sdpa, cuda_device, d):
     for b in range(B):  # rows past the length hold NaN: any read of them poisons O
         k[b, :, lens[b]:] = 0x7FC0
         v[b, :, lens[b]:] = 0x7FC0
-    scale = float(np.float32(1 / math.sqrt(d)))
+    # any finite scale: 0 averages the visible rows, a negative one flips the logits
+    scale = {"default": float(np.float32(1 / math.sqrt(d))), "zero": 0.0, "negative": -0.25}[scale_kind]
     tq, tk, tv = (W.to_torch(x, cuda_device) for x in (q, k, v))
     tl = torch.from_numpy(lens).to(cuda_device)
     o, lse = sdpa.decode(tq, tk, tv, tl, scale=scale)
     assert sdpa.get_last_device_error() == sdpa.SDPA_OK
     O_ref, L_ref = oracle.decode(si.bf16_bits_to_f32(q), si.bf16_bits_to_f32(k), si.bf16_bits_to_f32(v), lens, scale)
-    check_bf16(o.float().cpu().numpy().reshape(B * H, d), O_ref, lse.cpu().numpy().reshape(-1), L_ref, "decode d=%d" % d)
+    check_bf16(o.float().cpu().numpy().reshape(B * H, d), O_ref, lse.cpu().numpy().reshape(-1), L_ref,
+               "decode d=%d scale %g" % (d, scale))
 
 
 def test_decode_bad_length_reported(sdpa, cuda_device):
