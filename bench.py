@@ -406,8 +406,9 @@ def run_prefill_leg(args, sdpa, name, dev, stream, flush, peaks, peak_kind, cloc
 
 def run_backward(args, sdpa, si, W, name, dev, stream, flush, peaks, peak_kind, clocks):
     """dQ, dK, dV of a prefill workload from the forward's O and LSE.  Algorithmic FLOPs: 2.5x the
-    forward's (five matrix products of the gradient); the kernels execute 3.5x (S and dP are formed
-    in both the dK/dV and the dQ kernel)."""
+    forward's (five matrix products of the gradient).  At d = 64 the kernels execute exactly those
+    (dQ is formed beside dK and dV and reduce-added in fp32); at d = 128 they execute 3.5x (S and dP
+    are formed in both the dK/dV and the dQ kernel)."""
     import torch
     w = workload(name)
     inp = PrefillInputs(w, dev)
@@ -428,10 +429,11 @@ def run_backward(args, sdpa, si, W, name, dev, stream, flush, peaks, peak_kind, 
     t = float(per.mean())
     flops = 2.5 * w.flops()
     nbytes = 2 * w.bytes()  # Q, K, V, O, dO and LSE read; dQ, dK, dV written (dO is O's size)
-    roof = tensor_roofline("sdpa_bwd_pre + sdpa_bwd_dkdv + sdpa_bwd_dq (%s)" % name, flops, nbytes, t, peaks,
+    kernels = "sdpa_bwd_pre + sdpa_bwd_dkdv + %s" % ("sdpa_bwd_dq_out" if w.d == 64 else "sdpa_bwd_dq")
+    roof = tensor_roofline("%s (%s)" % (kernels, name), flops, nbytes, t, peaks,
                            peak_kind, profiled_traffic("backward_%s_dram.txt" % name, BWD_SOURCES),
                            "profiles/backward_%s_dram.txt (dK/dV and dQ kernels)" % name)
-    roof["executed_flop"] = 3.5 * w.flops()
+    roof["executed_flop"] = (2.5 if w.d == 64 else 3.5) * w.flops()
     return {"workload": DESCRIBE[name], "launches": n, "gpu_launches_per_call": 3, "ms": round(t * 1e3, 4),
             "value": round(flops / t / 1e12, 1), "unit": "TFLOP/s", "roofline": roof,
             "clocks": clocks.summary(t0, t1)}

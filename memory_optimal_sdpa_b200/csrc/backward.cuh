@@ -14,11 +14,17 @@
 //         S^T = K Q^T and dP^T = V dO^T (tcgen05, fp32 in TMEM), the elementwise
 //         P^T and dS^T (bf16, written back over S^T and dP^T), then dV += P^T dO and
 //         dK += dS^T Q with the TMEM operand form; dV and dK stay in TMEM to the end
+//   d = 64 (fused dQ): dkdv also writes dS^T into shared memory, forms dQ_t = dS_t K for each
+//         query tile t it visits (tcgen05, dS read as an MN-major operand, fp32 in TMEM) and
+//         reduce-adds it into an fp32 accumulator with a TMA reduce; then
+//   dq_out dQ = scale * accumulator in bf16.
+//   d = 128: dkdv's four accumulators fill TMEM, so dQ has its own kernel:
 //   dq    one CTA per 128-row query tile, streaming key tiles: S, dP, dS as above,
 //         then dQ += dS K; launched as a programmatic dependent of dkdv (which it does not
 //         read), so its CTAs fill the SMs dkdv's tail leaves
-// Each gradient is written once, so global traffic is O(n d) per kernel and no
-// atomics are needed; the price is computing S and dP in both kernels.
+// dK and dV are written once; dQ is written once at d = 128 (the price: S and dP formed in
+// both kernels) and accumulated in fp32 over the key tiles at d = 64 (S and dP formed once;
+// measured 425 -> 557 TF/s on 4 x 16 x 2048, 336 -> 420 causal).  Global traffic stays O(n d).
 //
 // Warp roles (384 threads, as the forward kernel): warps 0-7 two elementwise
 // warpgroups (warpgroup w takes columns [64 w, 64 w + 64) of the 128 x 128
@@ -42,6 +48,14 @@
 #define SDPA_BWD_DS_SEPARATE_D64 0  // measured: d = 64 backward 427 -> 414 TF/s with it, d = 128 709 -> 716
 #endif
 
+// d = 64: dQ is formed in the dK/dV kernel (dQ_t = dS_t K for each query tile t it visits, from dS
+// in shared memory) and reduce-added in fp32 into a workspace by TMA, so S and dP are computed
+// once instead of once per kernel; a small kernel then writes dQ in bf16.  At d = 128 the four
+// accumulators of the dK/dV kernel fill TMEM and leave no columns for dQ, so dQ keeps its own kernel.
+#ifndef SDPA_BWD_FUSED_DQ_D64
+#define SDPA_BWD_FUSED_DQ_D64 1
+#endif
+
 namespace sdpa {
 
 struct BwdParams {
@@ -53,6 +67,7 @@ struct BwdParams {
   __nv_bfloat16* dQ;        // [bh, n_q, D]
   __nv_bfloat16* dK;        // [bh, n_kv, D]
   __nv_bfloat16* dV;        // [bh, n_kv, D]
+  float* dQacc;             // [bh, n_q_pad, D] fp32 dQ / scale, reduce-added by the dK/dV kernel (fused dQ)
   int n_q, n_kv, n_q_pad, bh_count;
   float scale, scale_log2;
 };
@@ -61,17 +76,27 @@ template <int D>
 struct BwdCfg {
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int BLOCK_BYTES = 128 * 64 * 2;
-  // d = 64: four stages, which also keeps the CTA's shared memory above half an SM's, so a
-  // second CTA (that would wait for TMEM) is never placed beside it.
-  static constexpr int NSTAGE = (D == 64) ? 4 : 2;
+  // fused dQ (d = 64 only, see SDPA_BWD_FUSED_DQ_D64)
+  static constexpr bool FUSED_DQ = (D == 64) && SDPA_BWD_FUSED_DQ_D64;
+  // d = 64: four stages (three beside the fused dQ's buffers), which also keeps the CTA's shared
+  // memory above half an SM's, so a second CTA (that would wait for TMEM) is never placed beside it.
+  static constexpr int NSTAGE = (D == 64) ? (FUSED_DQ ? 3 : 4) : 2;
   static constexpr int VEC_BYTES = 1024;  // L2[128] then D[128] of a query tile (dkdv only)
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES + VEC_BYTES;
   static constexpr int FIX_OFF = 0;                // the CTA's fixed pair: (K, V) or (Q, dO)
   static constexpr int ST_OFF = 2 * TILE_BYTES;    // streamed stages: (Q, dO, vectors) or (K, V)
-  static constexpr int BAR_OFF = ST_OFF + NSTAGE * STAGE_BYTES;
+  // fused dQ: two buffers of dS^T (query tile t in buffer t % 2; bf16, 128 keys x 128 queries in
+  // two 64-query blocks, 128-byte swizzle), then the fp32 staging of dQ for the reduce (128 rows x
+  // 32 columns per elementwise warpgroup, 128-byte swizzle).  Warpgroup 0 stages in the fixed V
+  // tile's place: V is read once, into TMEM, before the first S product.
+  static constexpr int DS_BYTES = 128 * 128 * 2;
+  static constexpr int DS_OFF = ST_OFF + NSTAGE * STAGE_BYTES;
+  static constexpr int STG_OFF = DS_OFF + (FUSED_DQ ? 2 * DS_BYTES : 0);
+  static constexpr int STG_BYTES = 128 * 32 * 4;
+  static constexpr int BAR_OFF = STG_OFF + (FUSED_DQ ? STG_BYTES : 0);
   // fix_full, full[NSTAGE], empty[NSTAGE], s_full[2], p_full[2], grad_done[2], o_full, drain[2], fix_tmem,
-  // sd_free[2]
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 12;
+  // sd_free[2], dq_full, dq_free, ds_free[2]
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 12 + 4;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;
   static constexpr int THREADS = 384;
   static constexpr int EW_REGS = 192;  // 192 x 256 + 120 x 128 = 168 x 384: no spills in the control warps
@@ -96,6 +121,10 @@ struct BwdCfg {
   // S and dP, not until the dQ product has read dS.
   static constexpr bool DS_SEPARATE = SDPA_BWD_DS_SEPARATE_D64 || D == 128;
   static constexpr uint32_t COL_DS = FIX_IN_TMEM ? 448 : 384;
+  static constexpr uint32_t COL_DQ = 448;  // fused dQ: dQ_t (fp32, D columns) in the dK/dV kernel
+  static_assert(!FUSED_DQ || (FIX_IN_TMEM && !TWO_ISSUERS && COL_DQ + D <= TMEM_COLS && TILE_BYTES == STG_BYTES),
+                "fused dQ layout");
+  static_assert(DS_OFF % 1024 == 0 && STG_OFF % 1024 == 0, "swizzled buffers need 1 KB alignment");
 };
 
 // Programmatic dependent launch.  launch_dependents: the next kernel on the stream, if launched
@@ -121,6 +150,11 @@ __global__ void __launch_bounds__(128) sdpa_bwd_pre_kernel(const BwdParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e0 = (lane % LPR) * 8;
   const float POS_INF = __int_as_float(0x7f800000);
+  if (BwdCfg<D>::FUSED_DQ) {  // the fp32 dQ accumulator of these 128 rows starts at zero
+    float4* z = reinterpret_cast<float4*>(p.dQacc + ((size_t)bh * p.n_q_pad + r0) * D);
+#pragma unroll 4
+    for (int i = threadIdx.x; i < 128 * D / 4; i += 128) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   for (int it = 0; it < 128 / (4 * RPW); ++it) {
     const int row = r0 + (it * 4 + warp) * RPW + lane / LPR;
     float dot = 0.f;
@@ -148,6 +182,24 @@ __global__ void __launch_bounds__(128) sdpa_bwd_pre_kernel(const BwdParams p) {
         p.L2[o] = POS_INF;
       }
     }
+  }
+}
+
+// ------------------------------------------------------------------------------------ dQ out
+// Fused dQ: dQ = scale * dQacc in bf16, rows below n_q (eight elements per thread and pass).
+template <int D>
+__global__ void __launch_bounds__(256) sdpa_bwd_dq_out_kernel(const BwdParams p) {
+  const size_t n8 = (size_t)p.bh_count * p.n_q * (D / 8);
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n8; i += (size_t)gridDim.x * 256) {
+    const size_t row = i / (D / 8);  // bh * n_q + r
+    const int c = (int)(i % (D / 8)) * 8;
+    const size_t bh = row / p.n_q, r = row % p.n_q;
+    const float4* src = reinterpret_cast<const float4*>(p.dQacc + (bh * p.n_q_pad + r) * D + c);
+    const float4 a = src[0], b = src[1];
+    const float k = p.scale;
+    *reinterpret_cast<uint4*>(p.dQ + row * D + c) =
+        make_uint4(sm100::pack_bf16x2(a.x * k, a.y * k), sm100::pack_bf16x2(a.z * k, a.w * k),
+                   sm100::pack_bf16x2(b.x * k, b.y * k), sm100::pack_bf16x2(b.z * k, b.w * k));
   }
 }
 
@@ -179,7 +231,7 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     sdpa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                         const BwdParams p) {
+                         const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
   using C = BwdCfg<D>;
   using namespace sm100;
   // The dQ kernel after this one on the stream reads nothing it writes: once every CTA of this
@@ -200,6 +252,11 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* drain = o_full + 1;          // [issuer]
   uint64_t* fix_tmem = drain + 2;        // d = 64: the fixed pair has been copied into TMEM
   uint64_t* sd_free = fix_tmem + 1;      // [half] (dq): S and dP of half h are in registers
+  uint64_t* dq_full = sd_free + 2;       // fused dQ: dQ_t is in TMEM
+  uint64_t* dq_free = dq_full + 1;       // fused dQ: the elementwise warps have read dQ_t
+  uint64_t* ds_free = dq_free + 1;       // [buffer] fused dQ: the dQ_t product has read dS buffer t % 2
+  uint8_t* sDS = smem + C::DS_OFF;
+  uint8_t* sStg[2] = {sFix + C::TILE_BYTES, smem + C::STG_OFF};  // [warpgroup]
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -235,6 +292,10 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(fix_tmem, 256);
     mbar_init(&sd_free[0], 128);
     mbar_init(&sd_free[1], 128);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 256);
+    mbar_init(&ds_free[0], 1);
+    mbar_init(&ds_free[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -256,6 +317,7 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == C::LOAD_WARP) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0 && NT > 0) {
+        if (C::FUSED_DQ) tma_prefetch_desc(&tmdQacc);
         mbar_arrive_expect_tx(fix_full, 2 * C::TILE_BYTES);
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb) {
@@ -330,6 +392,19 @@ __global__ void __launch_bounds__(384, 1)
             mma_ts(tmem + C::COL_B, tmem + C::COL_DP + bwd_pair_col(kk), dQm + ob, idA, acc);
           }
         };
+        // fused dQ: dQ_t = dS_t K, this key tile's share of query tile t's dQ, fresh in TMEM.  A is
+        // dS (M = 128 queries, K = 128 keys) read MN-major from the buffer of dS^T rows (two
+        // 64-query blocks 16 KB apart); B is K (N = d, K = keys), MN-major like V in the forward.
+        constexpr uint32_t idQ = idesc_bf16_f32(128, D, true, true);
+        const uint64_t dKm = smem_desc_sw128(fix, C::BLOCK_BYTES, 1024);
+        auto issue_dq = [&](int t) {
+          const uint64_t dDSm = smem_desc_sw128(smem_u32(sDS + (t & 1) * C::DS_BYTES), C::BLOCK_BYTES, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            const uint64_t o = (uint64_t)((kk * 2048) >> 4);
+            mma_ss(tmem + C::COL_DQ, dDSm + o, dKm + o, idQ, kk > 0 ? 1u : 0u);
+          }
+        };
         // Half h of tile t + 1 starts as soon as warpgroup h has finished half h of tile t, so one
         // warpgroup's elementwise pass overlaps the other's and the tensor core's products.
         bool ok = true;
@@ -348,6 +423,12 @@ __global__ void __launch_bounds__(384, 1)
                 if (h == 0 && !(ok = wait_bar(&full[(t + 1) % C::NSTAGE], (t + 1) / C::NSTAGE))) break;
                 issue_sdp(t + 1, h);
               }
+            }
+            if (C::FUSED_DQ && ok) {  // both halves' dS_t are in the buffer; dQ_(t-1) has been read out
+              if (t > 0 && !(ok = wait_bar(dq_free, t - 1))) break;
+              issue_dq(t);
+              tc_commit(dq_full);
+              tc_commit(&ds_free[t & 1]);
             }
           }
           if (ok) tc_commit(o_full);
@@ -402,12 +483,47 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before_sync();
       mbar_arrive(fix_tmem);
     }
+    // Fused dQ: query tile tt's dQ_tt leaves TMEM through this warpgroup's staging buffer (its 32 of
+    // the D columns, rows = queries, 128-byte swizzle) and one TMA reduce-add into the fp32
+    // accumulator, issued by the warpgroup's first thread.  The warpgroup's four warps agree on
+    // every drain with a barrier vote, so a failed wait in any of them makes all of them skip it
+    // (and the later ones): each warp takes part in exactly NT votes, its share of every drain,
+    // whatever fails, and none is left waiting at a named barrier.
+    const int wg_bar = 1 + w;  // named barrier of this warpgroup (128 threads)
+    const bool wg_leader = (threadIdx.x & 127) == 0;
+    int n_votes = 0;
+    auto drain_dq = [&](int tt, bool can) -> bool {
+      const bool r = can && mbar_wait_bounded(dq_full, (uint32_t)tt & 1u, abort_flag, &timed_out);
+      if (wg_leader) bulk_wait_group_read_all();  // the previous reduce has read the staging buffer
+      ++n_votes;
+      if (named_bar_any(wg_bar, 128, !r)) return false;
+      tc_fence_after_sync();
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + C::COL_DQ + 32u * (uint32_t)w + lane_base, v);
+      tmem_wait_ld();
+      reg_fence(v);
+      tc_fence_before_sync();
+      mbar_arrive(dq_free);
+      uint8_t* rp = sStg[w] + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4)) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      fence_proxy_async_smem();
+      named_bar_sync(wg_bar, 128);
+      if (wg_leader) {
+        tma_reduce_add_3d(&tmdQacc, sStg[w], 32 * w, (t_first + tt) * 128, bh);
+        bulk_commit_group();
+      }
+      return true;
+    };
     for (int t = 0; ok && t < NT; ++t) {
       const int st = t % C::NSTAGE;
       const float* vL2 = reinterpret_cast<const float*>(sSt + st * C::STAGE_BYTES + 2 * C::TILE_BYTES);
       const float* vD = vL2 + 128;
       // the stage's vectors come from the bulk copy: wait for it here too, not only through the MMAs
       if (!(ok = wait_warp(&full[st], t / C::NSTAGE) && wait_warp(&s_full[w], t))) break;
+      // fused dQ: the dQ product of tile t - 2 has read dS buffer t % 2 (its (t / 2 - 1)-th use)
+      if (C::FUSED_DQ && t > 1 && !(ok = wait_warp(&ds_free[t & 1], t / 2 - 1))) break;
       tc_fence_after_sync();
       const int q0 = (t_first + t) * 128 + 64 * w;  // first query of this warpgroup's columns
       const bool masked = CAUSAL && (q0 + off < j0 + 127);
@@ -439,10 +555,25 @@ __global__ void __launch_bounds__(384, 1)
                           [&](int) { return true; }, pp, ps);
         tmem_st_32x32b_x16(tmem + C::COL_S + (uint32_t)(64 * w + 16 * h) + lane_base, pp);
         tmem_st_32x32b_x16(tmem + C::COL_DP + (uint32_t)(64 * w + 16 * h) + lane_base, ps);
+        if (C::FUSED_DQ) {  // and into the dS buffer: key `row`, this chunk's 32 queries (16-byte chunks 4h ..)
+          uint8_t* rp = sDS + (t & 1) * C::DS_BYTES + w * C::BLOCK_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4*>(rp + (((4 * h + i) ^ (row & 7)) << 4)) =
+                make_uint4(ps[4 * i], ps[4 * i + 1], ps[4 * i + 2], ps[4 * i + 3]);
+        }
       }
       tmem_wait_st();
       tc_fence_before_sync();
+      if (C::FUSED_DQ) fence_proxy_async_smem();  // the dS rows are read by the tensor core
       mbar_arrive(&p_full[w]);
+      if (C::FUSED_DQ && t > 0 && !(ok = drain_dq(t - 1, true))) break;
+    }
+    if (C::FUSED_DQ && NT > 0) {
+      // the last tile's dQ, then the votes a failure left out; all reduces complete before exit
+      if (n_votes < NT) ok = drain_dq(NT - 1, ok) && ok;
+      while (n_votes < NT) drain_dq(n_votes, false);
+      if (wg_leader) bulk_wait_group_all();
     }
     // ---------------------------------------------------------------- epilogue
     if (ok && NT > 0) ok = wait_warp(o_full, 0);

@@ -70,6 +70,22 @@ bool make_map(CUtensorMap* map, const void* ptr, int d, int n, int bh, int box_r
   return r == CUDA_SUCCESS;
 }
 
+// [bh][n][d] fp32 tensor, 32-column x 128-row boxes, 128-byte swizzle (the fused dQ accumulator).
+bool make_map_f32(CUtensorMap* map, const float* ptr, int d, int n, int bh) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)bh};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)n * d * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && debug_on())
+    std::fprintf(stderr, "sdpa: cuTensorMapEncodeTiled (fp32) failed (CUresult %d) d=%d n=%d bh=%d\n", (int)r, d, n, bh);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 // Multiprocessors of the current device (the persistent prefill grid).
@@ -488,44 +504,63 @@ template <int D, bool CAUSAL>
 int launch_bwd(const void* Q, const void* K, const void* V, const sdpa::BwdParams& p, cudaStream_t stream) {
   using Cfg = sdpa::BwdCfg<D>;
   auto kdkdv = sdpa::sdpa_bwd_dkdv_kernel<D, CAUSAL>;
-  auto kdq = sdpa::sdpa_bwd_dq_kernel<D, CAUSAL>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+    if constexpr (!Cfg::FUSED_DQ)
+      if (attr_err == cudaSuccess)
+        attr_err = cudaFuncSetAttribute(sdpa::sdpa_bwd_dq_kernel<D, CAUSAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        Cfg::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem, backward)", attr_err);
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdqa;
   if (!make_map(&mq, Q, D, p.n_q, p.bh_count) || !make_map(&mk, K, D, p.n_kv, p.bh_count) ||
       !make_map(&mv, V, D, p.n_kv, p.bh_count) || !make_map(&mdo, p.dO, D, p.n_q, p.bh_count))
     return SDPA_ERR_CUDA;
+  if (Cfg::FUSED_DQ) {
+    if (!make_map_f32(&mdqa, p.dQacc, D, p.n_q_pad, p.bh_count)) return SDPA_ERR_CUDA;
+  } else {
+    mdqa = mq;  // not read
+  }
   sdpa::sdpa_bwd_pre_kernel<D><<<dim3((unsigned)(p.n_q_pad / 128), (unsigned)p.bh_count), 128, 0, stream>>>(p);
   const long long n_kt = (p.n_kv + 127) / 128, n_qt = (p.n_q + 127) / 128;
-  kdkdv<<<(unsigned)(p.bh_count * n_kt), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
-  // dq reads only what the pre kernel wrote (complete before dkdv started), so it is launched as a
-  // programmatic dependent: its CTAs start on the SMs dkdv's last wave leaves, and it waits for
-  // dkdv itself before it completes.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(p.bh_count * n_qt));
-  cfg.blockDim = dim3(Cfg::THREADS);
-  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, kdq, mq, mk, mv, mdo, p);
-  return e == cudaSuccess ? SDPA_OK : cuda_fail("backward launch", e);
+  kdkdv<<<(unsigned)(p.bh_count * n_kt), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdqa, p);
+  if constexpr (Cfg::FUSED_DQ) {
+    // dQ = scale * the accumulator, in bf16 (eight elements per thread and pass)
+    const long long n8 = (long long)p.bh_count * p.n_q * (D / 8);
+    long long blocks = (n8 + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    sdpa::sdpa_bwd_dq_out_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SDPA_OK : cuda_fail("backward launch", e);
+  } else {
+    // dq reads only what the pre kernel wrote (complete before dkdv started), so it is launched as a
+    // programmatic dependent: its CTAs start on the SMs dkdv's last wave leaves, and it waits for
+    // dkdv itself before it completes.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.bh_count * n_qt));
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, sdpa::sdpa_bwd_dq_kernel<D, CAUSAL>, mq, mk, mv, mdo, p);
+    return e == cudaSuccess ? SDPA_OK : cuda_fail("backward launch", e);
+  }
 }
 }  // namespace
 
+// Per padded query row: D and LSE log2(e), then (used at d = 64) 64 fp32 dQ accumulator columns.
+constexpr long long kBwdFloatsPerRow = 2 + 64;
+
 extern "C" size_t sdpa_bwd_workspace_size(int batch, int heads, int n_q) {
   if (batch <= 0 || heads <= 0 || n_q <= 0) return 0;
-  return (size_t)(2LL * batch * heads * bwd_rows_padded(n_q)) * sizeof(float);
+  return (size_t)(kBwdFloatsPerRow * batch * heads * bwd_rows_padded(n_q)) * sizeof(float);
 }
 
 extern "C" int sdpa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
@@ -556,6 +591,7 @@ extern "C" int sdpa_bwd(const void* Q, const void* K, const void* V, const void*
   p.bh_count = (int)bh;
   p.Dvec = (float*)workspace;
   p.L2 = p.Dvec + (size_t)bh * p.n_q_pad;
+  p.dQacc = p.L2 + (size_t)bh * p.n_q_pad;  // 16-byte aligned: n_q_pad is a multiple of 128
   p.dQ = (__nv_bfloat16*)dQ;
   p.dK = (__nv_bfloat16*)dK;
   p.dV = (__nv_bfloat16*)dV;
