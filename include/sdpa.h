@@ -176,9 +176,10 @@ SDPA_API int sdpa_decode_noalloc(const void* Q, const void* K, const void* V, co
 
 /*
  * sdpa_bwd_workspace_size -- bytes of device workspace sdpa_bwd needs:
- * 66 * batch * heads * round_up(n_q, 128) floats: the per-row vectors D and LSE log2(e), and
- * 64 fp32 columns per row in which the d = 64 backward accumulates dQ before rounding it to bf16
- * (unused at d = 128).  0 for a degenerate shape.
+ * 74 * batch * heads * round_up(n_q, 128) floats: the per-row vectors D and LSE log2(e), then
+ * for the d = 64 backward 64 fp32 columns per row in which it accumulates dQ before rounding it
+ * to bf16, and 32 bytes per row of per-query terms it adds inside its tensor-core products
+ * (both unused at d = 128).  0 for a degenerate shape.
  */
 SDPA_API size_t sdpa_bwd_workspace_size(int batch, int heads, int n_q);
 

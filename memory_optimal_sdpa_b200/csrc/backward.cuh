@@ -68,6 +68,9 @@ struct BwdParams {
   __nv_bfloat16* dK;        // [bh, n_kv, D]
   __nv_bfloat16* dV;        // [bh, n_kv, D]
   float* dQacc;             // [bh, n_q_pad, D] fp32 dQ / scale, reduce-added by the dK/dV kernel (fused dQ)
+  // d = 64 kernel: per 128-row query tile, four 1 KB shared-memory images (8 rows x 64 queries bf16,
+  // 128-byte swizzle): -LSE log2(e) / (scale log2(e)) and -D of each half as three bf16 terms
+  uint8_t* aug;
   int n_q, n_kv, n_q_pad, bh_count;
   float scale, scale_log2;
 };
@@ -140,6 +143,22 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 // its 64 columns into [64 w, 64 w + 32) of the fp32 region it read them from.
 __device__ __forceinline__ uint32_t bwd_pair_col(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
 
+// v as hi + mid + lo, three bf16 values (round to nearest at each step; the remainders are exact
+// in fp32, so the sum carries v to 24 bits).  Infinite v: hi = v, mid = lo = 0.
+__device__ __forceinline__ void bwd_split3(float v, uint16_t (&t)[3]) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  t[0] = __bfloat16_as_ushort(hi);
+  if (!isfinite(v)) {
+    t[1] = t[2] = 0;
+    return;
+  }
+  const float r1 = v - __bfloat162float(hi);
+  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(mid);
+  t[1] = __bfloat16_as_ushort(mid);
+  t[2] = __bfloat16_as_ushort(__float2bfloat16_rn(r2));
+}
+
 // ------------------------------------------------------------------------------------ pre
 template <int D>
 __global__ void __launch_bounds__(128) sdpa_bwd_pre_kernel(const BwdParams p) {
@@ -150,7 +169,7 @@ __global__ void __launch_bounds__(128) sdpa_bwd_pre_kernel(const BwdParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e0 = (lane % LPR) * 8;
   const float POS_INF = __int_as_float(0x7f800000);
-  if (BwdCfg<D>::FUSED_DQ) {  // the fp32 dQ accumulator of these 128 rows starts at zero
+  if (D == 64 && p.dQacc) {  // the fp32 dQ accumulator of these 128 rows starts at zero
     float4* z = reinterpret_cast<float4*>(p.dQacc + ((size_t)bh * p.n_q_pad + r0) * D);
 #pragma unroll 4
     for (int i = threadIdx.x; i < 128 * D / 4; i += 128) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -181,6 +200,25 @@ __global__ void __launch_bounds__(128) sdpa_bwd_pre_kernel(const BwdParams p) {
         p.Dvec[o] = 0.f;
         p.L2[o] = POS_INF;
       }
+    }
+  }
+  if (D == 64 && p.aug) {
+    // The d = 64 kernel adds -LSE log2(e) / c2 to S and -D to dP inside the tensor-core products:
+    // each value as three bf16 terms (hi + mid + lo holds 24 bits) in rows 0-2 of a 64-query
+    // block, rows 3-7 zero, laid out as the kernel's shared memory expects.
+    __syncthreads();  // this block's D and LSE log2(e) values are written
+    const size_t o = (size_t)bh * p.n_q_pad + r0 + threadIdx.x;
+    const float vs = -p.L2[o] / p.scale_log2, vp = -p.Dvec[o];
+    uint16_t ts[3], tp[3];
+    bwd_split3(vs, ts);
+    bwd_split3(vp, tp);
+    const int h = threadIdx.x >> 6, col = threadIdx.x & 63;
+    uint16_t* img = reinterpret_cast<uint16_t*>(p.aug + ((size_t)bh * (p.n_q_pad / 128) + blockIdx.x) * 4096);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int e = (k * 128 + ((((col * 2) >> 4) ^ k) << 4) + ((col * 2) & 15)) >> 1;  // element within a 1 KB image
+      img[h * 512 + e] = k < 3 ? ts[k] : (uint16_t)0;
+      img[(2 + h) * 512 + e] = k < 3 ? tp[k] : (uint16_t)0;
     }
   }
 }

@@ -17,6 +17,7 @@
 #include "decode.cuh"
 #include "decode_gqa.cuh"
 #include "backward.cuh"
+#include "backward_d64.cuh"
 
 namespace {
 
@@ -555,8 +556,41 @@ int launch_bwd(const void* Q, const void* K, const void* V, const sdpa::BwdParam
 }
 }  // namespace
 
-// Per padded query row: D and LSE log2(e), then (used at d = 64) 64 fp32 dQ accumulator columns.
-constexpr long long kBwdFloatsPerRow = 2 + 64;
+// Per padded query row: D and LSE log2(e), then (used at d = 64) 64 fp32 dQ accumulator columns and
+// 32 bytes of the d = 64 kernel's per-query terms.
+constexpr long long kBwdFloatsPerRow = 2 + 64 + 8;
+
+// d = 64: the one-kernel backward (sdpa_bwd_d64_kernel), then dQ = scale * the fp32 accumulator.
+#ifndef SDPA_BWD_D64_KERNEL
+#define SDPA_BWD_D64_KERNEL 1
+#endif
+namespace {
+template <bool CAUSAL>
+int launch_bwd_d64(const void* Q, const void* K, const void* V, const sdpa::BwdParams& p, cudaStream_t stream) {
+  using Cfg = sdpa::BwdD64Cfg;
+  auto kern = sdpa::sdpa_bwd_d64_kernel<CAUSAL>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem, backward d64)", attr_err);
+  CUtensorMap mq, mk, mv, mdo, mdqa;
+  if (!make_map(&mq, Q, 64, p.n_q, p.bh_count) || !make_map(&mk, K, 64, p.n_kv, p.bh_count) ||
+      !make_map(&mv, V, 64, p.n_kv, p.bh_count) || !make_map(&mdo, p.dO, 64, p.n_q, p.bh_count) ||
+      !make_map_f32(&mdqa, p.dQacc, 64, p.n_q_pad, p.bh_count))
+    return SDPA_ERR_CUDA;
+  sdpa::sdpa_bwd_pre_kernel<64><<<dim3((unsigned)(p.n_q_pad / 128), (unsigned)p.bh_count), 128, 0, stream>>>(p);
+  const long long n_kt = (p.n_kv + 127) / 128;
+  kern<<<(unsigned)(p.bh_count * n_kt), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdqa, p);
+  const long long n8 = (long long)p.bh_count * p.n_q * (64 / 8);
+  long long blocks = (n8 + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  sdpa::sdpa_bwd_dq_out_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SDPA_OK : cuda_fail("backward launch", e);
+}
+}  // namespace
 
 extern "C" size_t sdpa_bwd_workspace_size(int batch, int heads, int n_q) {
   if (batch <= 0 || heads <= 0 || n_q <= 0) return 0;
@@ -591,15 +625,21 @@ extern "C" int sdpa_bwd(const void* Q, const void* K, const void* V, const void*
   p.bh_count = (int)bh;
   p.Dvec = (float*)workspace;
   p.L2 = p.Dvec + (size_t)bh * p.n_q_pad;
-  p.dQacc = p.L2 + (size_t)bh * p.n_q_pad;  // 16-byte aligned: n_q_pad is a multiple of 128
+  // d = 64 accumulates dQ in fp32 here (16-byte aligned: n_q_pad is a multiple of 128); its
+  // one-kernel form needs scale != 0 (it adds -LSE log2(e) / (scale log2(e)) to S)
+  p.dQacc = d_k == 64 ? p.L2 + (size_t)bh * p.n_q_pad : nullptr;
+  const bool one_kernel = d_k == 64 && SDPA_BWD_D64_KERNEL && std::fabs(scale * 1.4426950408889634f) >= 1e-30f;
+  p.aug = one_kernel && sdpa::BwdD64Cfg::AUG ? reinterpret_cast<uint8_t*>(p.dQacc + (size_t)bh * p.n_q_pad * 64) : nullptr;
   p.dQ = (__nv_bfloat16*)dQ;
   p.dK = (__nv_bfloat16*)dK;
   p.dV = (__nv_bfloat16*)dV;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = (cudaStream_t)stream;
-  if (d_k == 64)
+  if (d_k == 64) {
+    if (one_kernel) return causal ? launch_bwd_d64<true>(Q, K, V, p, s) : launch_bwd_d64<false>(Q, K, V, p, s);
     return causal ? launch_bwd<64, true>(Q, K, V, p, s) : launch_bwd<64, false>(Q, K, V, p, s);
+  }
   return causal ? launch_bwd<128, true>(Q, K, V, p, s) : launch_bwd<128, false>(Q, K, V, p, s);
 }
 

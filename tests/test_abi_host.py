@@ -152,8 +152,8 @@ def test_decode_gqa_workspace_and_errors(sdpa):
 def test_bwd_workspace_and_errors(sdpa):
     ws = sdpa.bwd_workspace_size
     assert ws(0, 1, 16) == 0 and ws(1, 1, 0) == 0
-    # D and LSE log2(e), plus 64 fp32 dQ accumulator columns, per row padded to a multiple of 128
-    assert ws(4, 16, 2048) == 66 * 4 * 16 * 2048 * 4 and ws(1, 2, 130) == 66 * 2 * 256 * 4
+    # D and LSE log2(e), 64 fp32 dQ accumulator columns and 8 words of per-query terms, per row padded to 128
+    assert ws(4, 16, 2048) == 74 * 4 * 16 * 2048 * 4 and ws(1, 2, 130) == 74 * 2 * 256 * 4
     d = sdpa.lib.sdpa_bwd
     need = ws(1, 2, 256)
     args = lambda **kw: dict(dict(Q=P, K=P, V=P, O=P, dO=P, L=P, dQ=P, dK=P, dV=P, b=1, h=2, nq=256, nkv=256, dk=64,
