@@ -49,7 +49,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SPEC = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 PREFILL_SOURCES = ["memory_optimal_sdpa_b200/csrc/prefill_bf16.cuh", "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
 DECODE_SOURCES = ["memory_optimal_sdpa_b200/csrc/decode.cuh"]
-BWD_SOURCES = ["memory_optimal_sdpa_b200/csrc/backward.cuh", "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
+BWD_SOURCES = ["memory_optimal_sdpa_b200/csrc/backward.cuh", "memory_optimal_sdpa_b200/csrc/backward_d64.cuh",
+               "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
 GQA_SOURCES = ["memory_optimal_sdpa_b200/csrc/decode_gqa.cuh", "memory_optimal_sdpa_b200/csrc/decode.cuh",
                "memory_optimal_sdpa_b200/csrc/sm100.cuh"]
 PREFILL_WORKLOADS = ["cfg4", "cfg3", "cfg2", "cfg2c", "cfg3w"]
@@ -429,10 +430,10 @@ def run_backward(args, sdpa, si, W, name, dev, stream, flush, peaks, peak_kind, 
     t = float(per.mean())
     flops = 2.5 * w.flops()
     nbytes = 2 * w.bytes()  # Q, K, V, O, dO and LSE read; dQ, dK, dV written (dO is O's size)
-    kernels = "sdpa_bwd_pre + sdpa_bwd_dkdv + %s" % ("sdpa_bwd_dq_out" if w.d == 64 else "sdpa_bwd_dq")
+    kernels = "sdpa_bwd_pre + " + ("sdpa_bwd_d64 + sdpa_bwd_dq_out" if w.d == 64 else "sdpa_bwd_dkdv + sdpa_bwd_dq")
     roof = tensor_roofline("%s (%s)" % (kernels, name), flops, nbytes, t, peaks,
                            peak_kind, profiled_traffic("backward_%s_dram.txt" % name, BWD_SOURCES),
-                           "profiles/backward_%s_dram.txt (dK/dV and dQ kernels)" % name)
+                           "profiles/backward_%s_dram.txt (all three kernels of a call)" % name)
     roof["executed_flop"] = (2.5 if w.d == 64 else 3.5) * w.flops()
     return {"workload": DESCRIBE[name], "launches": n, "gpu_launches_per_call": 3, "ms": round(t * 1e3, 4),
             "value": round(flops / t / 1e12, 1), "unit": "TFLOP/s", "roofline": roof,

@@ -19,16 +19,19 @@
 // more K step (see SDPA_BWD64_AUG), so the elementwise step is P = 2^(S' c2), dS = P dP' with no
 // per-column loads: those broadcast loads had cost about a fifth of the shared-memory bandwidth
 // (measured 4 x 16 x 2048: 507 -> 628 TF/s).
-// Warp roles (384 threads): warps 0-7 two elementwise warpgroups (warpgroup w takes query
+// Warp roles (512 threads): warps 0-7 two elementwise warpgroups (warpgroup w takes query
 // columns [64 w, 64 w + 64) of each tile: its "half"; thread = TMEM lane = key of the tile),
-// warp 8 the TMA producer, warp 9 the S / dP issuer and TMEM owner, warp 10 the issuer of the
-// gradient products (dV, dK, dQ), warp 11 idle.
+// warp 8 the TMA producer, warp 9 the issuer of S^T, dP^T and dQ and TMEM owner, warp 10 the
+// issuer of the dV and dK products, warp 11 idle, warps 12-15 the dQ drain (TMEM -> staging ->
+// TMA reduce-add).  Measured on 4 x 16 x 2048 (TF/s, non-causal / causal): dQ drained by the
+// elementwise warps with a two-stage ring 628 / 452; drain warpgroup and three stages 663-679 /
+// 474-489; dQ moved to the S issuer with N = 128 S^T, dP^T products 675 / 480.
 #pragma once
 
 #include "backward.cuh"
 
 #ifndef SDPA_BWD64_SDP_N128
-#define SDPA_BWD64_SDP_N128 0  // 1: S^T and dP^T of both halves in N = 128 products (measured slower: 575 vs 628 TF/s)
+#define SDPA_BWD64_SDP_N128 1  // S^T and dP^T of both halves in N = 128 products (half the instructions)
 #endif
 // The per-query terms enter the S^T and dP^T products as one more K = 16 step: A is a block of
 // ones (rows 0-2), B holds -LSE log2(e) / c2 and -D as three bf16 terms each (rows 0-2), so the
@@ -38,14 +41,29 @@
 #ifndef SDPA_BWD64_AUG
 #define SDPA_BWD64_AUG 1
 #endif
+// dQ_t leaves TMEM through a warpgroup of its own (warps 12-15, 512 threads) rather than through
+// the elementwise warps between two tiles.
+#ifndef SDPA_BWD64_DRAIN_WG
+#define SDPA_BWD64_DRAIN_WG 1
+#endif
+// The dQ products are issued by the S^T / dP^T issuer (after the next tile's S^T, dP^T) rather
+// than by the gradient issuer, which balances the two instruction streams (18 and 16 products).
+#ifndef SDPA_BWD64_DQ_ON_A
+#define SDPA_BWD64_DQ_ON_A 1
+#endif
 
 namespace sdpa {
 
 struct BwdD64Cfg {
   static constexpr int D = 64;
   static constexpr int TILE_BYTES = 128 * D * 2;  // one 128 x 64 bf16 tile = one 128-byte-swizzle block
-  static constexpr int NSTAGE = 2;
+  static constexpr bool DRAIN_WG = SDPA_BWD64_DRAIN_WG;
+  // Q_t, dO_t ring: three stages when the drain warpgroup stages dQ through one 16 KB image
+  static constexpr int NSTAGE = DRAIN_WG ? 3 : 2;
+  static constexpr int NSTG = DRAIN_WG ? 1 : 2;  // dQ staging images
   static constexpr bool AUG = SDPA_BWD64_AUG;
+  static constexpr bool SDP_N128 = SDPA_BWD64_SDP_N128;
+  static constexpr bool DQ_ON_A = SDPA_BWD64_DQ_ON_A;
   // per query tile after Q and dO: with AUG the four 1 KB images of the -LSE log2(e) / c2 and -D
   // terms ([S, dP] x [half]); else the vectors LSE log2(e) [128] and D [128]
   static constexpr int VEC_BYTES = AUG ? 4096 : 1024;
@@ -58,16 +76,20 @@ struct BwdD64Cfg {
   static constexpr int STG_OFF = DS_OFF + 2 * DS_BYTES;
   // AUG: the ones block (two 64-key images, rows 0-2 = 1) and 2 KB of zeros (rows 8-15 of every
   // augmented operand)
-  static constexpr int ONES_OFF = STG_OFF + 2 * STG_BYTES;
+  static constexpr int ONES_OFF = STG_OFF + NSTG * STG_BYTES;
   static constexpr int ZERO_OFF = ONES_OFF + (AUG ? 2048 : 0);
   static constexpr int BAR_OFF = ZERO_OFF + (AUG ? 2048 : 0);
   // fix_full, full[NSTAGE], empty[NSTAGE], s_full[2], sd_free[2], p_full[2], grad_done[2], o_full,
   // drain[2], dq_full, dq_free, ds_free[2], const_ready
   static constexpr int NBAR = 1 + 2 * NSTAGE + 8 + 1 + 2 + 4 + 1;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;
-  static constexpr int THREADS = 384;
-  static constexpr int EW_REGS = 192;  // 192 x 256 + 120 x 128 = 168 x 384
-  static constexpr int CONTROL_REGS = 120;
+  static constexpr int THREADS = DRAIN_WG ? 512 : 384;
+  static constexpr int LAUNCH_REGS = DRAIN_WG ? 128 : 168;  // registers per thread the launch provides
+  // 192 x 256 + 64 x 128 + 64 x 128 = 128 x 512 (without the drain warpgroup: 192 x 256 + 120 x 128 = 168 x 384)
+  static constexpr int EW_REGS = 192;
+  static constexpr int CONTROL_REGS = DRAIN_WG ? 64 : 120;
+  static constexpr int DRAIN_REGS = 64;
+  static constexpr int DRAIN_WARP0 = 12;
   static constexpr int LOAD_WARP = 8;
   static constexpr int SDP_WARP = 9;
   static constexpr int GRAD_WARP = 10;
@@ -127,7 +149,7 @@ __device__ __forceinline__ void bwd64_chunk_aug(const uint32_t* s, const uint32_
 }
 
 template <bool CAUSAL>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(BwdD64Cfg::THREADS, 1)
     sdpa_bwd_d64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                         const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
@@ -155,6 +177,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* const_ready = ds_free + 2;      // AUG: the ones and zero blocks are written
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  uint32_t* ds_count = tmem_slot + 2;  // DQ_ON_A: elementwise warps that have written their dS rows
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -182,13 +205,14 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&p_full[h], 128);
       mbar_init(&grad_done[h], 1);
       mbar_init(&drain[h], 1);
-      mbar_init(&ds_free[h], 1);
+      mbar_init(&ds_free[h], C::DQ_ON_A ? 2 : 1);  // the dK and dQ products of the buffer's tile
     }
     mbar_init(o_full, 1);
     mbar_init(dq_full, 1);
-    mbar_init(dq_free, 256);
+    mbar_init(dq_free, C::DRAIN_WG ? 128 : 256);
     mbar_init(const_ready, 256);
     *abort_flag = 0;
+    *ds_count = 0;
     fence_mbar_init();
   }
   if (warp == C::SDP_WARP) {
@@ -200,10 +224,60 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   bool timed_out = false;
-  static_assert(C::EW_REGS * 256 + C::CONTROL_REGS * 128 <= 168 * 384, "register split exceeds the launch");
+  static_assert(C::EW_REGS * 256 + C::CONTROL_REGS * 128 + (C::DRAIN_WG ? C::DRAIN_REGS * 128 : 0) <=
+                    C::LAUNCH_REGS * C::THREADS,
+                "register split exceeds the launch");
 
   const bool tmem_bad = tmem_alloc_bad(tmem);  // debug builds only
   if (tmem_bad) {
+  } else if (C::DRAIN_WG && warp >= C::DRAIN_WARP0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::DRAIN_REGS));
+    // ------------------------------------------------------------ dQ drain warpgroup
+    // dQ_t (TMEM lanes = the tile's queries, 64 fp32 columns), 32 columns at a time, through one
+    // staging image and a TMA reduce-add into the fp32 accumulator issued by the warpgroup's first
+    // thread.
+    // The four warps agree on every drain with a barrier vote (named barrier 3), so a failed wait
+    // in any of them makes all of them skip it and the later ones: each takes part in exactly NT
+    // votes whatever fails, and none is left at a named barrier.
+    const int row = 32 * (warp & 3) + lane;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const bool leader = threadIdx.x == 32 * C::DRAIN_WARP0;
+    int n_votes = 0;
+    auto drain = [&](int tt, bool can) -> bool {
+      const bool r = can && mbar_wait_bounded(dq_full, (uint32_t)tt & 1u, abort_flag, &timed_out);
+      if (leader) bulk_wait_group_read_all();  // the previous reduces have read the staging images
+      ++n_votes;
+      if (named_bar_any(3, 128, !r)) return false;
+      tc_fence_after_sync();
+      uint8_t* rp = sStg + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + C::COL_DQ + 32u * (uint32_t)c + lane_base, v);
+        tmem_wait_ld();
+        reg_fence(v);
+        if (c == 1) {  // dQ_t has left TMEM: the next dQ product may overwrite it
+          tc_fence_before_sync();
+          mbar_arrive(dq_free);
+          if (leader) bulk_wait_group_read_all();  // the first half's reduce has read the image
+          named_bar_sync(3, 128);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4*>(rp + ((k ^ (row & 7)) << 4)) = make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(3, 128);
+        if (leader) {
+          tma_reduce_add_3d(&tmdQacc, sStg, 32 * c, (t_first + tt) * 128, bh);
+          bulk_commit_group();
+        }
+      }
+      return true;
+    };
+    bool ok = true;
+    for (int t = 0; ok && t < NT; ++t) ok = drain(t, true);
+    while (n_votes < NT) drain(n_votes, false);
+    if (leader) bulk_wait_group_all();  // every reduce has completed before the CTA exits
   } else if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::CONTROL_REGS));
     if (warp == C::LOAD_WARP) {
@@ -249,10 +323,25 @@ __global__ void __launch_bounds__(384, 1)
         };
         const uint32_t fix = smem_u32(sFix), st0 = smem_u32(sSt), ds0 = smem_u32(sDS);
         bool ok = true;
+        // dQ_t = dS_t K (M = 128 queries, N = d, K = 128 keys): dS read MN-major from dS buffer t % 2
+        // (two 64-query blocks 16 KB apart), K MN-major like V in the forward.
+        constexpr uint32_t idQ = idesc_bf16_f32(128, 64, true, true);
+        const uint64_t dKm = smem_desc_sw128(fix, C::TILE_BYTES, 1024);
+        auto issue_dq = [&](int t) {
+          const uint64_t dSm = smem_desc_sw128(ds0 + (uint32_t)((t & 1) * C::DS_BYTES), C::TILE_BYTES, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t o = (uint64_t)((kk * 2048) >> 4);  // 16 keys
+            mma_ss(tmem + C::COL_DQ, dSm + o, dKm + o, idQ, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(dq_full);
+          tc_commit(&ds_free[t & 1]);
+        };
         if (role == 0) {
-          // S^T_h = K Q_h^T and dP^T_h = V dO_h^T (M = 128 keys, N = 64 queries of half h, K = d):
-          // K, V and the stage's Q, dO rows all K-major
-          constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
+          // S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = the tile's 128 queries or the 64 of
+          // half h, K = d): K, V and the stage's Q, dO rows all K-major.  With SDPA_BWD64_DQ_ON_A
+          // this issuer also forms dQ_(t-1) right after S^T, dP^T of tile t.
+          constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false), idS2 = idesc_bf16_f32(128, 128, false, false);
           const uint64_t dK = smem_desc_sw128(fix, 16, 1024), dV = smem_desc_sw128(fix + C::TILE_BYTES, 16, 1024);
           ok = wait_bar(fix_full, 0) && (!C::AUG || wait_bar(const_ready, 0));
           // AUG step: A = the ones block (M = 128 keys in two 64-key images 1 KB apart, MN-major),
@@ -261,57 +350,65 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t ones = smem_u32(smem + C::ONES_OFF), zero = smem_u32(smem + C::ZERO_OFF);
           const uint64_t dOnes = smem_desc_sw128(ones, 1024, zero - ones);
           auto aug_desc = [&](uint32_t img) { return smem_desc_sw128(img, 1024, zero - img); };
-          for (int t = 0; ok && SDPA_BWD64_SDP_N128 && t < NT; ++t) {
-            // one N = 128 product per operand step (both halves), after both halves of t - 1 are read
-            constexpr uint32_t idS2 = idesc_bf16_f32(128, 128, false, false);
+          // dS_t of both halves in shared memory (eight elementwise warps per tile: a count, since
+          // this issuer reads it up to a tile late) and dQ_(t-1) out of TMEM
+          auto dq_ready = [&](int t) {
+            bool r = count_wait_bounded(ds_count, 8u * (uint32_t)(t + 1), abort_flag, &timed_out);
+            if (r) tc_fence_after_sync();
+            if (r && t > 0) r = wait_bar(dq_free, t - 1);
+            return r;
+          };
+          for (int t = 0; ok && t < NT; ++t) {
             const int st = t % C::NSTAGE;
             if (!(ok = wait_bar(&full[st], t / C::NSTAGE))) break;
-            if (t > 0 && !(ok = wait_bar(&sd_free[0], t - 1) && wait_bar(&sd_free[1], t - 1))) break;
-            const uint32_t sq = st0 + st * C::STAGE_BYTES;
-            const uint64_t dQk = smem_desc_sw128(sq, 16, 1024), dOk = smem_desc_sw128(sq + C::TILE_BYTES, 16, 1024);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t o = (uint64_t)((kk * 32) >> 4);
-              mma_ss(tmem + C::COL_S, dK + o, dQk + o, idS2, kk > 0 ? 1u : 0u);
-              mma_ss(tmem + C::COL_DP, dV + o, dOk + o, idS2, kk > 0 ? 1u : 0u);
-            }
-            if (C::AUG) {  // images [S h0, S h1, dP h0, dP h1]: one N = 128 step each
-              const uint32_t img = sq + 2 * C::TILE_BYTES;
-              mma_ss(tmem + C::COL_S, dOnes, aug_desc(img), idAug2, 1u);
-              mma_ss(tmem + C::COL_DP, dOnes, aug_desc(img + 2048), idAug2, 1u);
-            }
-            tc_commit(&s_full[0]);
-            tc_commit(&s_full[1]);
-          }
-          for (int t = 0; ok && !SDPA_BWD64_SDP_N128 && t < NT; ++t) {
-            const int st = t % C::NSTAGE;
-            for (int h = 0; ok && h < 2; ++h) {
-              if (h == 0 && !(ok = wait_bar(&full[st], t / C::NSTAGE))) break;
-              if (t > 0 && !(ok = wait_bar(&sd_free[h], t - 1))) break;  // half h of tile t - 1 is in registers
-              const uint32_t sq = st0 + st * C::STAGE_BYTES + h * 8192;  // query rows 64 h ..
+            if (C::SDP_N128) {  // one N = 128 product per operand step, after both halves of t - 1 are read
+              if (t > 0 && !(ok = wait_bar(&sd_free[0], t - 1) && wait_bar(&sd_free[1], t - 1))) break;
+              const uint32_t sq = st0 + st * C::STAGE_BYTES;
               const uint64_t dQk = smem_desc_sw128(sq, 16, 1024), dOk = smem_desc_sw128(sq + C::TILE_BYTES, 16, 1024);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t o = (uint64_t)((kk * 32) >> 4);
-                mma_ss(tmem + C::COL_S + 64 * h, dK + o, dQk + o, idS, kk > 0 ? 1u : 0u);
-                mma_ss(tmem + C::COL_DP + 64 * h, dV + o, dOk + o, idS, kk > 0 ? 1u : 0u);
+                mma_ss(tmem + C::COL_S, dK + o, dQk + o, idS2, kk > 0 ? 1u : 0u);
+                mma_ss(tmem + C::COL_DP, dV + o, dOk + o, idS2, kk > 0 ? 1u : 0u);
               }
-              if (C::AUG) {
-                const uint32_t img = st0 + st * C::STAGE_BYTES + 2 * C::TILE_BYTES + h * 1024;
-                mma_ss(tmem + C::COL_S + 64 * h, dOnes, aug_desc(img), idAug1, 1u);
-                mma_ss(tmem + C::COL_DP + 64 * h, dOnes, aug_desc(img + 2048), idAug1, 1u);
+              if (C::AUG) {  // images [S h0, S h1, dP h0, dP h1]: one N = 128 step each
+                const uint32_t img = sq + 2 * C::TILE_BYTES;
+                mma_ss(tmem + C::COL_S, dOnes, aug_desc(img), idAug2, 1u);
+                mma_ss(tmem + C::COL_DP, dOnes, aug_desc(img + 2048), idAug2, 1u);
               }
-              tc_commit(&s_full[h]);
+              tc_commit(&s_full[0]);
+              tc_commit(&s_full[1]);
+            } else {
+              for (int h = 0; ok && h < 2; ++h) {
+                if (t > 0 && !(ok = wait_bar(&sd_free[h], t - 1))) break;  // half h of tile t - 1 is in registers
+                const uint32_t sq = st0 + st * C::STAGE_BYTES + h * 8192;  // query rows 64 h ..
+                const uint64_t dQk = smem_desc_sw128(sq, 16, 1024), dOk = smem_desc_sw128(sq + C::TILE_BYTES, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t o = (uint64_t)((kk * 32) >> 4);
+                  mma_ss(tmem + C::COL_S + 64 * h, dK + o, dQk + o, idS, kk > 0 ? 1u : 0u);
+                  mma_ss(tmem + C::COL_DP + 64 * h, dV + o, dOk + o, idS, kk > 0 ? 1u : 0u);
+                }
+                if (C::AUG) {
+                  const uint32_t img = st0 + st * C::STAGE_BYTES + 2 * C::TILE_BYTES + h * 1024;
+                  mma_ss(tmem + C::COL_S + 64 * h, dOnes, aug_desc(img), idAug1, 1u);
+                  mma_ss(tmem + C::COL_DP + 64 * h, dOnes, aug_desc(img + 2048), idAug1, 1u);
+                }
+                tc_commit(&s_full[h]);
+              }
+              if (!ok) break;
+            }
+            if (C::DQ_ON_A && t > 0) {
+              if (!(ok = dq_ready(t - 1))) break;
+              issue_dq(t - 1);
             }
           }
+          if (C::DQ_ON_A && ok && (ok = dq_ready(NT - 1))) issue_dq(NT - 1);
         } else {
           // dV += P^T_h dO_h (A = P^T from TMEM), dK += dS^T_h Q_h (A = dS^T K-major from shared
           // memory), M = 128 keys, N = d, K = the 64 queries of half h; dO_h, Q_h MN-major.  Then
-          // dQ_t = dS_t K (M = 128 queries, N = d, K = 128 keys): dS read MN-major from the same
-          // buffer (two 64-query blocks 16 KB apart), K MN-major.
+          // (without SDPA_BWD64_DQ_ON_A) dQ_t.
           constexpr uint32_t idG = idesc_bf16_f32(128, 64, false, true);
-          constexpr uint32_t idQ = idesc_bf16_f32(128, 64, true, true);
-          const uint64_t dKm = smem_desc_sw128(fix, C::TILE_BYTES, 1024);
           for (int t = 0; ok && t < NT; ++t) {
             const int st = t % C::NSTAGE;
             const uint32_t sq = st0 + st * C::STAGE_BYTES;
@@ -328,18 +425,16 @@ __global__ void __launch_bounds__(384, 1)
                 mma_ss(tmem + C::COL_DK, dSk + (uint64_t)((k4 * 32) >> 4), dQm + ob, idG, acc);
               }
               tc_commit(&grad_done[h]);
-              if (h == 1) tc_commit(&empty[st]);
+              if (h == 1) {
+                tc_commit(&empty[st]);
+                if (C::DQ_ON_A) tc_commit(&ds_free[t & 1]);  // with the S issuer's commit after dQ_t
+              }
             }
             if (!ok) break;
-            if (t > 0 && !(ok = wait_bar(dq_free, t - 1))) break;  // dQ_(t-1) has left TMEM
-            const uint64_t dSm = smem_desc_sw128(dsb, C::TILE_BYTES, 1024);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t o = (uint64_t)((kk * 2048) >> 4);  // 16 keys
-              mma_ss(tmem + C::COL_DQ, dSm + o, dKm + o, idQ, kk > 0 ? 1u : 0u);
+            if (!C::DQ_ON_A) {
+              if (t > 0 && !(ok = wait_bar(dq_free, t - 1))) break;  // dQ_(t-1) has left TMEM
+              issue_dq(t);
             }
-            tc_commit(dq_full);
-            tc_commit(&ds_free[t & 1]);
           }
           if (ok) tc_commit(o_full);
         }
@@ -454,9 +549,13 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before_sync();
       fence_proxy_async_smem();  // the dS^T rows are read by the tensor core
       mbar_arrive(&p_full[w]);
-      if (t > 0 && !(ok = drain_dq(t - 1, true))) break;
+      if (C::DQ_ON_A) {
+        __syncwarp();
+        if (lane == 0) red_release_add(ds_count, 1u);
+      }
+      if (!C::DRAIN_WG && t > 0 && !(ok = drain_dq(t - 1, true))) break;
     }
-    if (NT > 0) {
+    if (!C::DRAIN_WG && NT > 0) {
       // the last tile's dQ, then the votes a failure left out; all reduces complete before exit
       if (n_votes < NT) ok = drain_dq(NT - 1, ok) && ok;
       while (n_votes < NT) drain_dq(n_votes, false);
