@@ -56,6 +56,13 @@
 #define SDPA_BWD_FUSED_DQ_D64 1
 #endif
 
+// d = 128 dK/dV kernel: the per-query terms -LSE log2(e) / c2 and -D enter the S^T and dP^T products
+// as one more K = 16 step against a block of ones (as in the d = 64 kernel), so the elementwise
+// step reads no per-column vectors; used when the host supplies the term images (scale != 0).
+#ifndef SDPA_BWD_AUG_D128
+#define SDPA_BWD_AUG_D128 1
+#endif
+
 namespace sdpa {
 
 struct BwdParams {
@@ -84,7 +91,10 @@ struct BwdCfg {
   // d = 64: four stages (three beside the fused dQ's buffers), which also keeps the CTA's shared
   // memory above half an SM's, so a second CTA (that would wait for TMEM) is never placed beside it.
   static constexpr int NSTAGE = (D == 64) ? (FUSED_DQ ? 3 : 4) : 2;
-  static constexpr int VEC_BYTES = 1024;  // L2[128] then D[128] of a query tile (dkdv only)
+  static constexpr bool AUG = (D == 128) && SDPA_BWD_AUG_D128;
+  // dkdv, per query tile after Q and dO: L2[128] then D[128], or (AUG) the four 1 KB images of the
+  // per-query terms ([S, dP] x [half])
+  static constexpr int VEC_BYTES = AUG ? 4096 : 1024;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES + VEC_BYTES;
   static constexpr int FIX_OFF = 0;                // the CTA's fixed pair: (K, V) or (Q, dO)
   static constexpr int ST_OFF = 2 * TILE_BYTES;    // streamed stages: (Q, dO, vectors) or (K, V)
@@ -96,10 +106,13 @@ struct BwdCfg {
   static constexpr int DS_OFF = ST_OFF + NSTAGE * STAGE_BYTES;
   static constexpr int STG_OFF = DS_OFF + (FUSED_DQ ? 2 * DS_BYTES : 0);
   static constexpr int STG_BYTES = 128 * 32 * 4;
-  static constexpr int BAR_OFF = STG_OFF + (FUSED_DQ ? STG_BYTES : 0);
+  // AUG: the ones block (two 64-key images, rows 0-2 = 1) and 2 KB of zeros
+  static constexpr int ONES_OFF = STG_OFF + (FUSED_DQ ? STG_BYTES : 0);
+  static constexpr int ZERO_OFF = ONES_OFF + (AUG ? 2048 : 0);
+  static constexpr int BAR_OFF = ZERO_OFF + (AUG ? 2048 : 0);
   // fix_full, full[NSTAGE], empty[NSTAGE], s_full[2], p_full[2], grad_done[2], o_full, drain[2], fix_tmem,
-  // sd_free[2], dq_full, dq_free, ds_free[2]
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 12 + 4;
+  // sd_free[2], dq_full, dq_free, ds_free[2], const_ready
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 12 + 5;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;
   static constexpr int THREADS = 384;
   static constexpr int EW_REGS = 192;  // 192 x 256 + 120 x 128 = 168 x 384: no spills in the control warps
@@ -127,7 +140,10 @@ struct BwdCfg {
   static constexpr uint32_t COL_DQ = 448;  // fused dQ: dQ_t (fp32, D columns) in the dK/dV kernel
   static_assert(!FUSED_DQ || (FIX_IN_TMEM && !TWO_ISSUERS && COL_DQ + D <= TMEM_COLS && TILE_BYTES == STG_BYTES),
                 "fused dQ layout");
-  static_assert(DS_OFF % 1024 == 0 && STG_OFF % 1024 == 0, "swizzled buffers need 1 KB alignment");
+  static_assert(DS_OFF % 1024 == 0 && STG_OFF % 1024 == 0 && ONES_OFF % 1024 == 0 && ZERO_OFF % 1024 == 0 &&
+                    STAGE_BYTES % 1024 == 0,
+                "swizzled buffers need 1 KB alignment");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 // Programmatic dependent launch.  launch_dependents: the next kernel on the stream, if launched
@@ -202,8 +218,8 @@ __global__ void __launch_bounds__(128) sdpa_bwd_pre_kernel(const BwdParams p) {
       }
     }
   }
-  if (D == 64 && p.aug) {
-    // The d = 64 kernel adds -LSE log2(e) / c2 to S and -D to dP inside the tensor-core products:
+  if (p.aug) {
+    // The d = 64 kernel and the d = 128 dK/dV kernel add -LSE log2(e) / c2 to S and -D to dP inside the tensor-core products:
     // each value as three bf16 terms (hi + mid + lo holds 24 bits) in rows 0-2 of a 64-query
     // block, rows 3-7 zero, laid out as the kernel's shared memory expects.
     __syncthreads();  // this block's D and LSE log2(e) values are written
@@ -293,6 +309,9 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* dq_full = sd_free + 2;       // fused dQ: dQ_t is in TMEM
   uint64_t* dq_free = dq_full + 1;       // fused dQ: the elementwise warps have read dQ_t
   uint64_t* ds_free = dq_free + 1;       // [buffer] fused dQ: the dQ_t product has read dS buffer t % 2
+  uint64_t* const_ready = ds_free + 2;   // AUG: the ones and zero blocks are written
+  // AUG at run time: the host supplied the per-query term images (it does when scale != 0)
+  const bool aug = C::AUG && p.aug != nullptr;
   uint8_t* sDS = smem + C::DS_OFF;
   uint8_t* sStg[2] = {sFix + C::TILE_BYTES, smem + C::STG_OFF};  // [warpgroup]
   uint32_t* tmem_slot = (uint32_t*)(bars + C::NBAR);
@@ -334,6 +353,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(dq_free, 256);
     mbar_init(&ds_free[0], 1);
     mbar_init(&ds_free[1], 1);
+    mbar_init(const_ready, 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -368,15 +388,20 @@ __global__ void __launch_bounds__(384, 1)
           if (!mbar_wait_bounded(&empty[st], ((uint32_t)(t / C::NSTAGE) & 1u) ^ 1u, abort_flag, &timed_out)) break;
           uint8_t* dst = sSt + st * C::STAGE_BYTES;
           const int q0 = (t_first + t) * 128;
-          mbar_arrive_expect_tx(&full[st], 2 * C::TILE_BYTES + C::VEC_BYTES);
+          mbar_arrive_expect_tx(&full[st], 2 * C::TILE_BYTES + (aug ? 4096 : 1024));
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb) {
             tma_load_3d(dst + cb * C::BLOCK_BYTES, &tmQ, &full[st], cb * 64, q0, bh);
             tma_load_3d(dst + C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmdO, &full[st], cb * 64, q0, bh);
           }
-          const size_t v0 = (size_t)bh * p.n_q_pad + q0;
-          bulk_load(dst + 2 * C::TILE_BYTES, p.L2 + v0, 512, &full[st]);
-          bulk_load(dst + 2 * C::TILE_BYTES + 512, p.Dvec + v0, 512, &full[st]);
+          if (aug) {
+            bulk_load(dst + 2 * C::TILE_BYTES, p.aug + ((size_t)bh * (p.n_q_pad / 128) + (t_first + t)) * 4096, 4096,
+                      &full[st]);
+          } else {
+            const size_t v0 = (size_t)bh * p.n_q_pad + q0;
+            bulk_load(dst + 2 * C::TILE_BYTES, p.L2 + v0, 512, &full[st]);
+            bulk_load(dst + 2 * C::TILE_BYTES + 512, p.Dvec + v0, 512, &full[st]);
+          }
           issued = t + 1;
         }
         if (*abort_flag) {  // let the copies in flight land before the CTA exits
@@ -415,6 +440,14 @@ __global__ void __launch_bounds__(384, 1)
               mma_ss(tmem + C::COL_DP + 64 * h, dV + o, dOk + o, idS, kk > 0 ? 1u : 0u);
             }
           }
+          if (aug) {  // + ones x the half's term images (S: images 0, 1; dP: images 2, 3), MN-major
+            const uint32_t img = st0 + (t % C::NSTAGE) * C::STAGE_BYTES + 2 * C::TILE_BYTES + h * 1024;
+            const uint32_t ones = smem_u32(smem + C::ONES_OFF), zero = smem_u32(smem + C::ZERO_OFF);
+            const uint64_t dOnes = smem_desc_sw128(ones, 1024, zero - ones);
+            constexpr uint32_t idAug = idesc_bf16_f32(128, 64, true, true);
+            mma_ss(tmem + C::COL_S + 64 * h, dOnes, smem_desc_sw128(img, 1024, zero - img), idAug, 1u);
+            mma_ss(tmem + C::COL_DP + 64 * h, dOnes, smem_desc_sw128(img + 2048, 1024, zero - img - 2048), idAug, 1u);
+          }
           tc_commit(&s_full[h]);
         };
         auto issue_grad = [&](int t, int h) {  // dV += P^T_h dO_h, dK += dS^T_h Q_h (64 query rows)
@@ -447,7 +480,8 @@ __global__ void __launch_bounds__(384, 1)
         // warpgroup's elementwise pass overlaps the other's and the tensor core's products.
         bool ok = true;
         if (!C::TWO_ISSUERS) {
-          ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0) && (!C::FIX_IN_TMEM || wait_bar(fix_tmem, 0));
+          ok = wait_bar(fix_full, 0) && wait_bar(&full[0], 0) && (!C::FIX_IN_TMEM || wait_bar(fix_tmem, 0)) &&
+               (!aug || wait_bar(const_ready, 0));
           if (ok) {
             issue_sdp(0, 0);
             issue_sdp(0, 1);
@@ -471,7 +505,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           if (ok) tc_commit(o_full);
         } else if (role == 0) {  // S / dP: half h of tile t once the gradient products of half h of t - 1 are done
-          ok = wait_bar(fix_full, 0) && (!C::FIX_IN_TMEM || wait_bar(fix_tmem, 0));
+          ok = wait_bar(fix_full, 0) && (!C::FIX_IN_TMEM || wait_bar(fix_tmem, 0)) && (!aug || wait_bar(const_ready, 0));
           for (int t = 0; ok && t < NT; ++t)
             for (int h = 0; ok && h < 2; ++h) {
               if (h == 0 && !(ok = wait_bar(&full[t % C::NSTAGE], t / C::NSTAGE))) break;
@@ -521,6 +555,16 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before_sync();
       mbar_arrive(fix_tmem);
     }
+    if (aug) {  // the ones block (rows 0-2 of both 64-key images) and the zeros, 16 bytes per thread
+      const int i = threadIdx.x;  // 0 .. 255
+      const uint32_t one2 = 0x3F803F80u;  // two bf16 ones
+      const bool ones_row = i < 128 && ((i & 63) >> 3) < 3;  // byte (i & 63) * 16 of image i >> 6: row (i & 63) / 8
+      *reinterpret_cast<uint4*>(smem + C::ONES_OFF + i * 16) =
+          ones_row ? make_uint4(one2, one2, one2, one2) : make_uint4(0u, 0u, 0u, 0u);
+      if (i >= 128) *reinterpret_cast<uint4*>(smem + C::ZERO_OFF + (i - 128) * 16) = make_uint4(0u, 0u, 0u, 0u);
+      fence_proxy_async_smem();
+      mbar_arrive(const_ready);
+    }
     // Fused dQ: query tile tt's dQ_tt leaves TMEM through this warpgroup's staging buffer (its 32 of
     // the D columns, rows = queries, 128-byte swizzle) and one TMA reduce-add into the fp32
     // accumulator, issued by the warpgroup's first thread.  The warpgroup's four warps agree on
@@ -559,7 +603,8 @@ __global__ void __launch_bounds__(384, 1)
       const float* vL2 = reinterpret_cast<const float*>(sSt + st * C::STAGE_BYTES + 2 * C::TILE_BYTES);
       const float* vD = vL2 + 128;
       // the stage's vectors come from the bulk copy: wait for it here too, not only through the MMAs
-      if (!(ok = wait_warp(&full[st], t / C::NSTAGE) && wait_warp(&s_full[w], t))) break;
+      // (with the term images in the products nothing of the stage is read here)
+      if (!(ok = (aug || wait_warp(&full[st], t / C::NSTAGE)) && wait_warp(&s_full[w], t))) break;
       // fused dQ: the dQ product of tile t - 2 has read dS buffer t % 2 (its (t / 2 - 1)-th use)
       if (C::FUSED_DQ && t > 1 && !(ok = wait_warp(&ds_free[t & 1], t / 2 - 1))) break;
       tc_fence_after_sync();
@@ -576,21 +621,29 @@ __global__ void __launch_bounds__(384, 1)
         reg_fence(dp);
         uint32_t pp[16], ps[16];
         const int qc = q0 + 32 * h;
-        // this chunk's 32 query vectors, four per 16-byte load (every lane reads the same words)
-        float l2v[32], ddv[32];
+        if (C::AUG && aug) {  // the per-query terms are already in s and dp
+          const auto zero = [](int) { return 0.f; };
+          if (masked)
+            bwd_elementwise(s, dp, c2, zero, zero, [&](int c) { return key <= qc + c + off; }, pp, ps);
+          else
+            bwd_elementwise(s, dp, c2, zero, zero, [&](int) { return true; }, pp, ps);
+        } else {
+          // this chunk's 32 query vectors, four per 16-byte load (every lane reads the same words)
+          float l2v[32], ddv[32];
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          const float4 a = *reinterpret_cast<const float4*>(vL2 + cbase + c);
-          const float4 b = *reinterpret_cast<const float4*>(vD + cbase + c);
-          l2v[c] = a.x, l2v[c + 1] = a.y, l2v[c + 2] = a.z, l2v[c + 3] = a.w;
-          ddv[c] = b.x, ddv[c + 1] = b.y, ddv[c + 2] = b.z, ddv[c + 3] = b.w;
+          for (int c = 0; c < 32; c += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(vL2 + cbase + c);
+            const float4 b = *reinterpret_cast<const float4*>(vD + cbase + c);
+            l2v[c] = a.x, l2v[c + 1] = a.y, l2v[c + 2] = a.z, l2v[c + 3] = a.w;
+            ddv[c] = b.x, ddv[c + 1] = b.y, ddv[c + 2] = b.z, ddv[c + 3] = b.w;
+          }
+          if (masked)
+            bwd_elementwise(s, dp, c2, [&](int c) { return l2v[c]; }, [&](int c) { return ddv[c]; },
+                            [&](int c) { return key <= qc + c + off; }, pp, ps);
+          else
+            bwd_elementwise(s, dp, c2, [&](int c) { return l2v[c]; }, [&](int c) { return ddv[c]; },
+                            [&](int) { return true; }, pp, ps);
         }
-        if (masked)
-          bwd_elementwise(s, dp, c2, [&](int c) { return l2v[c]; }, [&](int c) { return ddv[c]; },
-                          [&](int c) { return key <= qc + c + off; }, pp, ps);
-        else
-          bwd_elementwise(s, dp, c2, [&](int c) { return l2v[c]; }, [&](int c) { return ddv[c]; },
-                          [&](int) { return true; }, pp, ps);
         tmem_st_32x32b_x16(tmem + C::COL_S + (uint32_t)(64 * w + 16 * h) + lane_base, pp);
         tmem_st_32x32b_x16(tmem + C::COL_DP + (uint32_t)(64 * w + 16 * h) + lane_base, ps);
         if (C::FUSED_DQ) {  // and into the dS buffer: key `row`, this chunk's 32 queries (16-byte chunks 4h ..)

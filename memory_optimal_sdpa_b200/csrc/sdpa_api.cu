@@ -629,7 +629,10 @@ extern "C" int sdpa_bwd(const void* Q, const void* K, const void* V, const void*
   // one-kernel form needs scale != 0 (it adds -LSE log2(e) / (scale log2(e)) to S)
   p.dQacc = d_k == 64 ? p.L2 + (size_t)bh * p.n_q_pad : nullptr;
   const bool one_kernel = d_k == 64 && SDPA_BWD_D64_KERNEL && std::fabs(scale * 1.4426950408889634f) >= 1e-30f;
-  p.aug = one_kernel && sdpa::BwdD64Cfg::AUG ? reinterpret_cast<uint8_t*>(p.dQacc + (size_t)bh * p.n_q_pad * 64) : nullptr;
+  // the per-query term images (d = 64 one-kernel form; d = 128 dK/dV kernel), both need scale != 0
+  const bool terms = std::fabs(scale * 1.4426950408889634f) >= 1e-30f &&
+                     (d_k == 64 ? one_kernel && sdpa::BwdD64Cfg::AUG : sdpa::BwdCfg<128>::AUG);
+  p.aug = terms ? reinterpret_cast<uint8_t*>(p.L2 + (size_t)bh * p.n_q_pad * 65) : nullptr;
   p.dQ = (__nv_bfloat16*)dQ;
   p.dK = (__nv_bfloat16*)dK;
   p.dV = (__nv_bfloat16*)dV;
