@@ -581,8 +581,10 @@ int launch_bwd_d64(const void* Q, const void* K, const void* V, const sdpa::BwdP
       !make_map_f32(&mdqa, p.dQacc, 64, p.n_q_pad, p.bh_count))
     return SDPA_ERR_CUDA;
   sdpa::sdpa_bwd_pre_kernel<64><<<dim3((unsigned)(p.n_q_pad / 128), (unsigned)p.bh_count), 128, 0, stream>>>(p);
-  const long long n_kt = (p.n_kv + 127) / 128;
-  kern<<<(unsigned)(p.bh_count * n_kt), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdqa, p);
+  // persistent: one CTA per SM (at most one per unit), each walking (batch-head, key tile) units
+  long long grid = (long long)p.bh_count * ((p.n_kv + 127) / 128);
+  if (grid > sm_count()) grid = sm_count();
+  kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdqa, p);
   const long long n8 = (long long)p.bh_count * p.n_q * (64 / 8);
   long long blocks = (n8 + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;
@@ -631,7 +633,7 @@ extern "C" int sdpa_bwd(const void* Q, const void* K, const void* V, const void*
   const bool one_kernel = d_k == 64 && SDPA_BWD_D64_KERNEL && std::fabs(scale * 1.4426950408889634f) >= 1e-30f;
   // the per-query term images (d = 64 one-kernel form; d = 128 dK/dV kernel), both need scale != 0
   const bool terms = std::fabs(scale * 1.4426950408889634f) >= 1e-30f &&
-                     (d_k == 64 ? one_kernel && sdpa::BwdD64Cfg::AUG : sdpa::BwdCfg<128>::AUG);
+                     (d_k == 64 ? one_kernel : sdpa::BwdCfg<128>::AUG);
   p.aug = terms ? reinterpret_cast<uint8_t*>(p.L2 + (size_t)bh * p.n_q_pad * 65) : nullptr;
   p.dQ = (__nv_bfloat16*)dQ;
   p.dK = (__nv_bfloat16*)dK;
