@@ -38,18 +38,26 @@
 
 #include "backward.cuh"
 
+// K, V buffers: 1 reloads them in place after the unit's last product reading them (with three
+// Q/dO stages); 2 lets the next unit's K and V load during the current unit, but leaves room for
+// two stages only (measured 4 x 16 x 2048: 720 -> 648 TF/s, causal 515 -> 468).
+#ifndef SDPA_BWD64_KV_BUFFERS
+#define SDPA_BWD64_KV_BUFFERS 1
+#endif
+
 namespace sdpa {
 
 struct BwdD64Cfg {
   static constexpr int D = 64;
   static constexpr int TILE_BYTES = 128 * D * 2;  // one 128 x 64 bf16 tile = one 128-byte-swizzle block
-  static constexpr int NSTAGE = 3;                // Q_t, dO_t ring
+  static constexpr int NFIX = SDPA_BWD64_KV_BUFFERS;  // K, V buffers
+  static constexpr int NSTAGE = NFIX == 2 ? 2 : 3;     // Q_t, dO_t ring
   static constexpr int TERM_BYTES = 4096;         // the four 1 KB term images ([S, dP] x [half])
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES + TERM_BYTES;
   static constexpr int DS_BYTES = 128 * 128 * 2;
   static constexpr int STG_BYTES = 128 * 32 * 4;
-  static constexpr int FIX_OFF = 0;  // K, V
-  static constexpr int ST_OFF = 2 * TILE_BYTES;
+  static constexpr int FIX_OFF = 0;  // [buffer] K, V
+  static constexpr int ST_OFF = NFIX * 2 * TILE_BYTES;
   static constexpr int DS_OFF = ST_OFF + NSTAGE * STAGE_BYTES;
   static constexpr int STG_OFF = DS_OFF + 2 * DS_BYTES;
   // the ones block (two 64-key images, rows 0-2 = 1) and 2 KB of zeros (rows 8-15 of every
@@ -57,9 +65,9 @@ struct BwdD64Cfg {
   static constexpr int ONES_OFF = STG_OFF + STG_BYTES;
   static constexpr int ZERO_OFF = ONES_OFF + 2048;
   static constexpr int BAR_OFF = ZERO_OFF + 2048;
-  // fix_full, fix_free, full[NSTAGE], empty[NSTAGE], s_full[2], sd_free[2], p_full[2], grad_done[2],
-  // o_full, drain[2], dq_full, dq_free, ds_free[2], const_ready
-  static constexpr int NBAR = 2 + 2 * NSTAGE + 8 + 1 + 2 + 4 + 1;
+  // fix_full[NFIX], fix_free[NFIX], full[NSTAGE], empty[NSTAGE], s_full[2], sd_free[2], p_full[2],
+  // grad_done[2], o_full, drain[2], dq_full, dq_free, ds_free[2], const_ready
+  static constexpr int NBAR = 2 * NFIX + 2 * NSTAGE + 8 + 1 + 2 + 4 + 1;
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 16 + 1024;
   static constexpr int THREADS = 512;
   static constexpr int LAUNCH_REGS = 128;  // registers per thread the launch provides
@@ -108,14 +116,14 @@ __global__ void __launch_bounds__(BwdD64Cfg::THREADS, 1)
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sFix = smem + C::FIX_OFF;  // K, V
+  uint8_t* sFix = smem + C::FIX_OFF;  // [buffer] K, V
   uint8_t* sSt = smem + C::ST_OFF;    // per stage: Q, dO, the term images
   uint8_t* sDS = smem + C::DS_OFF;    // [tile % 2] dS^T
   uint8_t* sStg = smem + C::STG_OFF;  // dQ staging
   uint64_t* bars = (uint64_t*)(smem + C::BAR_OFF);
-  uint64_t* fix_full = bars;                // K, V of a unit landed (one phase per unit with tiles)
-  uint64_t* fix_free = fix_full + 1;        // the unit's last product reading K, V completed
-  uint64_t* full = fix_free + 1;            // [stage]
+  uint64_t* fix_full = bars;                // [buffer] K, V of a unit landed (units with tiles, in turn)
+  uint64_t* fix_free = fix_full + C::NFIX;  // [buffer] the unit's last product reading K, V completed
+  uint64_t* full = fix_free + C::NFIX;      // [stage]
   uint64_t* empty = full + C::NSTAGE;       // [stage]
   uint64_t* s_full = empty + C::NSTAGE;     // [half]: S^T and dP^T of the half are in TMEM
   uint64_t* sd_free = s_full + 2;           // [half]: ... and in the elementwise warps' registers
@@ -159,8 +167,10 @@ __global__ void __launch_bounds__(BwdD64Cfg::THREADS, 1)
   };
 
   if (threadIdx.x == 0) {
-    mbar_init(fix_full, 1);
-    mbar_init(fix_free, 1);
+    for (int i = 0; i < C::NFIX; ++i) {
+      mbar_init(&fix_full[i], 1);
+      mbar_init(&fix_free[i], 1);
+    }
     for (int i = 0; i < C::NSTAGE; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
@@ -262,11 +272,14 @@ __global__ void __launch_bounds__(BwdD64Cfg::THREADS, 1)
         for (int k = 0, u = unit_of(0), g = 0; ok && u < n_units; u = unit_of(++k)) {
           const Unit U = unit_at(u);
           if (U.NT == 0) continue;
-          // K, V replace the previous unit's once its last S^T, dP^T and dQ products have run
-          if (nf > 0 && !(ok = mbar_wait_bounded(fix_free, (uint32_t)(nf - 1) & 1u, abort_flag, &timed_out))) break;
-          mbar_arrive_expect_tx(fix_full, 2 * C::TILE_BYTES);
-          tma_load_3d(sFix, &tmK, fix_full, 0, U.j0, U.bh);
-          tma_load_3d(sFix + C::TILE_BYTES, &tmV, fix_full, 0, U.j0, U.bh);
+          // K, V replace those of the unit NFIX units back once its last S^T, dP^T and dQ products have run
+          const int b = nf % C::NFIX;
+          if (nf >= C::NFIX &&
+              !(ok = mbar_wait_bounded(&fix_free[b], (uint32_t)(nf / C::NFIX - 1) & 1u, abort_flag, &timed_out)))
+            break;
+          mbar_arrive_expect_tx(&fix_full[b], 2 * C::TILE_BYTES);
+          tma_load_3d(sFix + b * 2 * C::TILE_BYTES, &tmK, &fix_full[b], 0, U.j0, U.bh);
+          tma_load_3d(sFix + b * 2 * C::TILE_BYTES + C::TILE_BYTES, &tmV, &fix_full[b], 0, U.j0, U.bh);
           ++nf;
           for (int t = 0; t < U.NT; ++t) {
             const int gi = g + t, st = gi % C::NSTAGE;
@@ -284,7 +297,8 @@ __global__ void __launch_bounds__(BwdD64Cfg::THREADS, 1)
           g += U.NT;
         }
         if (*abort_flag) {  // let the copies in flight land before the CTA exits
-          if (nf > 0) mbar_wait_drain(fix_full, (uint32_t)(nf - 1) & 1u);
+          for (int i = (nf > C::NFIX ? nf - C::NFIX : 0); i < nf; ++i)
+            mbar_wait_drain(&fix_full[i % C::NFIX], (uint32_t)(i / C::NFIX) & 1u);
           for (int gi = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); gi < issued; ++gi)
             mbar_wait_drain(&full[gi % C::NSTAGE], (uint32_t)(gi / C::NSTAGE) & 1u);
         }
@@ -306,13 +320,12 @@ __global__ void __launch_bounds__(BwdD64Cfg::THREADS, 1)
           // in two 64-key images 1 KB apart, MN-major), B = the tile's term images (N = queries,
           // MN-major), rows 8-15 of both read the zeros.
           constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false), idT = idesc_bf16_f32(128, 128, true, true);
-          const uint64_t dK = smem_desc_sw128(fix, 16, 1024), dV = smem_desc_sw128(fix + C::TILE_BYTES, 16, 1024);
+          uint64_t dK = 0, dV = 0, dKm = 0;  // this unit's K, V buffer (set per unit)
           const uint32_t ones = smem_u32(smem + C::ONES_OFF), zero = smem_u32(smem + C::ZERO_OFF);
           const uint64_t dOnes = smem_desc_sw128(ones, 1024, zero - ones);
           // dQ_t = dS_t K (M = 128 queries, N = d, K = 128 keys): dS read MN-major from dS buffer
           // t % 2 (two 64-query blocks 16 KB apart), K MN-major like V in the forward.
           constexpr uint32_t idQ = idesc_bf16_f32(128, 64, true, true);
-          const uint64_t dKm = smem_desc_sw128(fix, C::TILE_BYTES, 1024);
           // dQ_gi may be formed once both halves' dS_gi are in shared memory (eight elementwise
           // warps per tile: a count, since this issuer reads it up to a tile late) and dQ_(gi-1)
           // has left TMEM
@@ -335,7 +348,12 @@ __global__ void __launch_bounds__(BwdD64Cfg::THREADS, 1)
           for (int k = 0, u = unit_of(0), g = 0, nf = 0; ok && u < n_units; u = unit_of(++k)) {
             const Unit U = unit_at(u);
             if (U.NT == 0) continue;
-            if (!(ok = wait_bar(fix_full, nf))) break;
+            const int b = nf % C::NFIX;
+            if (!(ok = wait_bar(&fix_full[b], nf / C::NFIX))) break;
+            const uint32_t kv = fix + (uint32_t)(b * 2 * C::TILE_BYTES);
+            dK = smem_desc_sw128(kv, 16, 1024);
+            dV = smem_desc_sw128(kv + C::TILE_BYTES, 16, 1024);
+            dKm = smem_desc_sw128(kv, C::TILE_BYTES, 1024);
             for (int t = 0; ok && t < U.NT; ++t) {
               const int gi = g + t, st = gi % C::NSTAGE;
               if (!(ok = wait_bar(&full[st], gi / C::NSTAGE))) break;
@@ -358,7 +376,7 @@ __global__ void __launch_bounds__(BwdD64Cfg::THREADS, 1)
             }
             // the unit's last dQ, then K and V may be replaced
             if (!ok || !(ok = issue_dq(g + U.NT - 1))) break;
-            tc_commit(fix_free);
+            tc_commit(&fix_free[b]);
             g += U.NT;
             ++nf;
           }

@@ -227,3 +227,26 @@ def test_bwd_zero_and_negative_scale(sdpa, cuda_device, B, H, n_q, n_kv, d, caus
                         dof[b, h], scale, causal, tag)
     if scale == 0.0:
         assert (dq == 0).all() and (dk == 0).all()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("scale,std", [(1e-3, 1.0), (None, 2.5)])
+def test_bwd_extreme_logit_ranges(sdpa, cuda_device, d, causal, scale, std):
+    # The tensor-core backward adds -LSE log2(e) / (scale log2(e)) to S inside the S product, as
+    # three bf16 terms: a tiny scale makes that term large against S (about 1e4 here), and wide
+    # inputs (N(0, 2.5^2), the 1 x 8 x 32768 workload's distribution) make the softmax sharp.
+    # Both must stay within the same per-element bounds as the ordinary cases.
+    B, H, n = 1, 2, 320
+    seed = 950 + d + int(causal) + (0 if scale is None else 7)
+    q = si.fill_host((B, H, n, d), seed, 0, b=std)
+    k = si.fill_host((B, H, n, d), seed, 1, b=std)
+    v = si.fill_host((B, H, n, d), seed, 2)
+    do = si.fill_host((B, H, n, d), seed, si.STREAM_DO)
+    scale = float(np.float32(1 / math.sqrt(d) if scale is None else scale))
+    dq, dk, dv = run_bwd(sdpa, cuda_device, q, k, v, do, causal, scale)
+    qf, kf, vf, dof = (si.bf16_bits_to_f32(x) for x in (q, k, v, do))
+    dQ, dK, dV = oracle.sdpa_backward(qf, kf, vf, dof, scale, causal)
+    for h in range(H):
+        check_slice(dq[0, h], dk[0, h], dv[0, h], dQ[0, h], dK[0, h], dV[0, h], qf[0, h], kf[0, h], vf[0, h],
+                    dof[0, h], scale, causal, "d=%d causal=%s scale=%g std=%g h=%d" % (d, causal, scale, std, h))
