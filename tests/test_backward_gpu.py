@@ -250,3 +250,29 @@ def test_bwd_extreme_logit_ranges(sdpa, cuda_device, d, causal, scale, std):
     for h in range(H):
         check_slice(dq[0, h], dk[0, h], dv[0, h], dQ[0, h], dK[0, h], dV[0, h], qf[0, h], kf[0, h], vf[0, h],
                     dof[0, h], scale, causal, "d=%d causal=%s scale=%g std=%g h=%d" % (d, causal, scale, std, h))
+
+
+def _random_shapes(count, seed):
+    # seeded shapes: ragged lengths on both sides, both head dims, both masks, several heads
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(count):
+        out.append((1, int(rng.integers(1, 4)), int(rng.integers(1, 600)), int(rng.integers(1, 600)),
+                    int(rng.choice([64, 128])), bool(rng.integers(0, 2))))
+    return out
+
+
+@pytest.mark.parametrize("B,H,n_q,n_kv,d,causal", _random_shapes(12, 2024))
+def test_bwd_random_shapes(sdpa, cuda_device, B, H, n_q, n_kv, d, causal):
+    seed = 1300 + 7 * n_q + 3 * n_kv + d + int(causal)
+    q = si.fill_host((B, H, n_q, d), seed, 0)
+    k = si.fill_host((B, H, n_kv, d), seed, 1)
+    v = si.fill_host((B, H, n_kv, d), seed, 2)
+    do = si.fill_host((B, H, n_q, d), seed, si.STREAM_DO)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    dq, dk, dv = run_bwd(sdpa, cuda_device, q, k, v, do, causal, scale)
+    qf, kf, vf, dof = (si.bf16_bits_to_f32(x) for x in (q, k, v, do))
+    dQ, dK, dV = oracle.sdpa_backward(qf, kf, vf, dof, scale, causal)
+    for h in range(H):
+        check_slice(dq[0, h], dk[0, h], dv[0, h], dQ[0, h], dK[0, h], dV[0, h], qf[0, h], kf[0, h], vf[0, h],
+                    dof[0, h], scale, causal, "%s h=%d" % ((B, H, n_q, n_kv, d, causal), h))

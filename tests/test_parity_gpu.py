@@ -333,6 +333,25 @@ def test_prefill_window_small(sdpa, cuda_device, B, H, n_q, n_kv, d, left, right
     assert torch.isnan(o_flat[o.numel():]).all() and torch.isnan(l_flat[lse.numel():]).all()
 
 
+
+def _random_window_shapes(count, seed):
+    # seeded shapes: ragged lengths, both head dims, windows from a single key to wider than the
+    # sequence, either side open (-1)
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(count):
+        n_q, n_kv = int(rng.integers(1, 700)), int(rng.integers(1, 700))
+        side = lambda: int(rng.choice([-1, 0, int(rng.integers(1, 300)), 1000]))
+        out.append((1, int(rng.integers(1, 4)), n_q, n_kv, int(rng.choice([64, 128])), side(), side()))
+    return out
+
+
+@pytest.mark.parametrize("B,H,n_q,n_kv,d,left,right", _random_window_shapes(14, 77))
+def test_prefill_window_random_shapes(sdpa, cuda_device, B, H, n_q, n_kv, d, left, right):
+    # the full, causal and windowed kernels all sit behind sdpa_fwd_window (open sides pick the
+    # plain instantiations), so random windows cover every mask mode on ragged shapes
+    test_prefill_window_small(sdpa, cuda_device, B, H, n_q, n_kv, d, left, right)
+
 def test_window_open_sides_equal_plain_calls(sdpa, cuda_device):
     import torch
     B, H, n, d = 1, 2, 640, 128
