@@ -190,7 +190,10 @@ SDPA_API size_t sdpa_bwd_workspace_size(int batch, int heads, int n_q);
  *
  * With P = softmax(Q K^T scale) recomputed from LSE, D_i = dO_i . O_i and dS = P (dO V^T - D):
  *   dV = P^T dO,   dK = scale dS^T Q,   dQ = scale dS K.
- * Nothing of size n_q x n_kv is written; each gradient is written once.
+ * Nothing of size n_q x n_kv is written; each gradient is written once.  At d = 64 (scale != 0)
+ * dQ is first summed over the key tiles in fp32 in the workspace by reduce-adds whose order is not
+ * fixed, so dQ can differ in its last bits from one call to the next (dK and dV, and everything
+ * at d = 128, are reproducible).
  * Q, O, dO, dQ [batch, heads, n_q, d]; K, V, dK, dV [batch, heads, n_kv, d]; all
  * __nv_bfloat16, contiguous, 16-byte aligned.  LSE [batch, heads, n_q] float as sdpa_fwd wrote
  * it (required).  d_k == d_v in {64, 128}; scale (any finite value) and causal as in the forward call.
