@@ -128,8 +128,11 @@ def test_decode_gqa_workspace_and_errors(sdpa):
     ws = sdpa.decode_gqa_workspace_size
     assert ws(0, 8, 1, 16, 128) == 0 and ws(1, 6, 4, 16, 128) == 0 and ws(1, 8, 0, 16, 128) == 0
     # 64 batches x 64 query heads over 8 key/value heads, 16384-row cache, d = 128 (tensor-core
-    # path): 2048-key splits, 8 per head, each d_v + 1 floats per query head
-    assert ws(64, 64, 8, 16384, 128) == 64 * 64 * 8 * 129 * 4
+    # path): 4096-key splits, 4 per head, each d_v + 1 floats per query head
+    assert ws(64, 64, 8, 16384, 128) == 64 * 64 * 4 * 129 * 4
+    # few (batch, group) pairs: the split halves until the grid has 4 CTAs per SM or reaches 128
+    # keys (1 x 8 groups over a 16384-row cache: 128-key splits, 128 per group)
+    assert ws(1, 64, 8, 16384, 128) == 1 * 64 * 128 * 129 * 4
     # group size one is plain decode and sizes like it
     assert ws(64, 32, 32, 16384, 128) == sdpa.decode_workspace_size(64, 32, 16384, 128)
     d = sdpa.lib.sdpa_decode_gqa
