@@ -18,6 +18,8 @@
 //         query tile t it visits (tcgen05, dS read as an MN-major operand, fp32 in TMEM) and
 //         reduce-adds it into an fp32 accumulator with a TMA reduce; then
 //   dq_out dQ = scale * accumulator in bf16.
+//         (At d = 64 with scale != 0 the host runs the one-kernel form of backward_d64.cuh
+//         instead; this fused path serves scale 0.)
 //   d = 128: dkdv's four accumulators fill TMEM, so dQ has its own kernel:
 //   dq    one CTA per 128-row query tile, streaming key tiles: S, dP, dS as above,
 //         then dQ += dS K; launched as a programmatic dependent of dkdv (which it does not
