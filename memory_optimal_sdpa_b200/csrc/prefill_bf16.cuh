@@ -599,11 +599,15 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive(&s_free[x]);
         }
         const int kv0 = (first + j) * 128;
-        const bool masked = kv0 + 127 > lim || kv0 < lo;
+        // Modes 0 and 1 have lo = 0, which kv0 + c >= 0 never falls below: one compare per score.
+        const bool masked = kv0 + 127 > lim || (MASK == 2 && kv0 < lo);
+        // With two exponential loops (d = 64) the loop is chosen per warp: a row of a masked tile
+        // may itself see every key, and two loops in one warp would run one after the other.
+        const bool warp_masked = C::POLY_EVERY > 0 ? __any_sync(0xffffffffu, masked) : masked;
         if (masked) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (kv0 + c > lim || kv0 + c < lo) s[c] = __float_as_uint(NEG_INF);
+            if (kv0 + c > lim || (MASK == 2 && kv0 + c < lo)) s[c] = __float_as_uint(NEG_INF);
         }
         float mx;
         {  // eight independent chains of 3-input maxima over s[0..127]: 16 + 7 x 16 scores
@@ -648,7 +652,7 @@ __global__ void __launch_bounds__(384, 1)
         if (SDPA_SM_TURN && !(ok = turn_wait())) break;  // this warp's turn on the exponentials
         const float m_use = (m_u == NEG_INF) ? 0.f : m_u;
         uint32_t pk[64];
-        l += masked ? softmax_exp_row<0>(s, c2, m_use, pk) : softmax_exp_row<C::POLY_EVERY>(s, c2, m_use, pk);
+        l += warp_masked ? softmax_exp_row<0>(s, c2, m_use, pk) : softmax_exp_row<C::POLY_EVERY>(s, c2, m_use, pk);
         if (SDPA_SM_TURN) turn_pass();  // hand the exponentials over
         if (C::P_SEPARATE && rx + j > 0 && !pv_waited) {  // the last P_x V (this unit's or the previous one's) reads P_x
           if (!(ok = wait_warp(&pv_done[x], rx + j - 1))) break;
