@@ -18,9 +18,12 @@
 //   warp  11   idle
 // Registers: each SM sub-partition holds 16K 32-bit registers and receives
 // one warp of every warpgroup, so the CTA launches at 168 per thread and then
-// moves registers from the producer/MMA warpgroup (down to 72) to the two
-// softmax warpgroups (up to 216): 2*216 + 72 <= 512 per sub-partition lane
-// slot, and 72*128 + 216*256 = 384*168 in total.
+// moves registers from the producer/MMA warpgroup to the two softmax
+// warpgroups: d = 64 72 and 216 (2*216 + 72 <= 512 per sub-partition lane slot,
+// 72*128 + 216*256 = 384*168 in total), d = 128 88 and 208 (the same totals),
+// where the MMA issuers' shared-S bookkeeping spills at 72 and the softmax
+// still fits in 208 (measured: 1 x 32 x 8192 with a 512-key window 533 -> 561
+// TF/s, the others unchanged or within noise; at d = 64 the 216 pays, by 1 %).
 //
 // TMEM (512 columns).  d = 64: S_a [0,128), S_b [128,256), P_a [256,320),
 // P_b [320,384), O_a [384,448), O_b [448,512).  With P in its own columns the
@@ -73,8 +76,8 @@ struct PrefillCfg {
   static constexpr int SMEM_BYTES = BAR_OFF + NBAR * 8 + 48 + 1024;
   static_assert(4 + 4 + 8 * 4 + 4 <= 48, "words after the barriers");
   static constexpr int THREADS = 384;
-  static constexpr int SOFTMAX_REGS = 216;
-  static constexpr int CONTROL_REGS = 72;
+  static constexpr int SOFTMAX_REGS = (D == 128) ? 208 : 216;
+  static constexpr int CONTROL_REGS = (D == 128) ? 88 : 72;
   static constexpr int LOAD_WARP = 8;
   static constexpr int MMA_WARP = 9;
   static constexpr uint32_t TMEM_COLS = 512;
