@@ -608,9 +608,26 @@ __global__ void __launch_bounds__(384, 1)
         // may itself see every key, and two loops in one warp would run one after the other.
         const bool warp_masked = C::POLY_EVERY > 0 ? __any_sync(0xffffffffu, masked) : masked;
         if (masked) {
+          if (MASK == 2) {
+            // Two-sided: per 32-column chunk, one mask of the hidden columns (below lo or above
+            // lim), then a bit test and a select per score.
+            const int hi = lim - kv0, lw = lo - kv0;  // this row sees columns lw .. hi
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (kv0 + c > lim || (MASK == 2 && kv0 + c < lo)) s[c] = __float_as_uint(NEG_INF);
+            for (int q = 0; q < 4; ++q) {
+              const int nb = min(max(lw - 32 * q, 0), 32);      // columns [0, nb) of the chunk are below lo
+              const int na = min(max(hi - 32 * q + 1, 0), 32);  // columns [na, 32) are above lim
+              const uint32_t below = nb >= 32 ? 0xffffffffu : (1u << nb) - 1u;
+              const uint32_t kept = na >= 32 ? 0xffffffffu : (1u << na) - 1u;
+              const uint32_t hidden = below | ~kept;
+#pragma unroll
+              for (int b = 0; b < 32; ++b)
+                if (hidden & (1u << b)) s[32 * q + b] = __float_as_uint(NEG_INF);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (kv0 + c > lim) s[c] = __float_as_uint(NEG_INF);
+          }
         }
         float mx;
         {  // eight independent chains of 3-input maxima over s[0..127]: 16 + 7 x 16 scores
